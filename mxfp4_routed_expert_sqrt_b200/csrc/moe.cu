@@ -1,0 +1,290 @@
+// libmoe.so: the C ABI declared in include/moe.h.  One translation unit: the
+// kernels live in the headers included below.
+#include <cstdio>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+moe_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "libmoe: launch failed: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status check_dims(const moe_dims* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->hidden <= 0 || d->inter <= 0 || d->n_experts <= 0 || d->top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (d->hidden % 32 || d->inter % 32) return MOE_ERR_UNSUPPORTED;
+  if (!pow2(d->hidden / 32) || !pow2(d->inter / 32) || d->hidden / 32 > 128 || d->inter / 32 > 128)
+    return MOE_ERR_UNSUPPORTED;
+  if (d->n_experts > 1024 || d->top_k > 32 || d->top_k > d->n_experts) return MOE_ERR_UNSUPPORTED;
+  if (!(d->swiglu_limit > 0.f) || !(d->swiglu_limit <= 32.f)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_proj(const moe_mxfp4_proj& p, int rows, int cols) {
+  if (p.base == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p.rows != rows || p.cols != cols) return MOE_ERR_INVALID_ARG;
+  if (p.expert_bytes != (int64_t)rows * cols / 2 + (int64_t)rows * cols / 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(p.base, 32) || p.expert_bytes % 16) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+// ---- GEMV launch ----------------------------------------------------------
+
+template <int WF, int P, int RBI, int NTP>
+moe_status launch_gemv_inst(const GemvArgs& a, cudaStream_t s) {
+  auto kern = gemv_kernel<WF, P, RBI, NTP>;
+  const int64_t row_bytes = gemv_row_bytes(WF, a.a.cols);
+  const int64_t stage = ((int64_t)P * a.rb * row_bytes + 127) / 128 * 128;
+  const int smem = (int)(stage * kGemvStages);
+  static bool configured = false;  // per instantiation; the attribute is per function
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = true;
+  }
+  kern<<<sm_count(), kGemvThreads, smem, s>>>(a);
+  return launch_status();
+}
+
+// Rows per unit: RBI * rp, with the largest RBI in {16, 8, 4, 2, 1} whose
+// stage fits the byte target and whose row block divides the rows, keeping
+// the scale block a multiple of 16 bytes.
+template <int WF, int P, int NTP>
+moe_status launch_gemv(GemvArgs a, cudaStream_t s) {
+  const int gpr = a.a.cols / 32, rp = kGemvThreads / gpr;
+  const int64_t row_bytes = gemv_row_bytes(WF, a.a.cols);
+  for (int rbi = 16; rbi >= 1; rbi >>= 1) {
+    const int rb = rbi * rp;
+    if (a.a.rows % rb) continue;
+    if (rbi > 1 && (int64_t)P * rb * row_bytes > kGemvStageTarget) continue;
+    if (WF == kWMxfp4 && ((int64_t)rb * (a.a.cols / 32)) % 16) continue;
+    const int seg = gpr < 32 ? gpr : 32;
+    if ((kGemvThreads / seg) * P * rbi * NTP > kGemvRedFloats) continue;
+    a.rb = rb;
+    switch (rbi) {
+      case 16: return launch_gemv_inst<WF, P, 16, NTP>(a, s);
+      case 8: return launch_gemv_inst<WF, P, 8, NTP>(a, s);
+      case 4: return launch_gemv_inst<WF, P, 4, NTP>(a, s);
+      case 2: return launch_gemv_inst<WF, P, 2, NTP>(a, s);
+      default: return launch_gemv_inst<WF, P, 1, NTP>(a, s);
+    }
+  }
+  return MOE_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_ALIGNMENT: return "misaligned pointer or size";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+int32_t moe_device_error(void) {
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error, sizeof(v)) != cudaSuccess) return -1;
+  if (cudaMemcpyToSymbol(g_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  return v;
+}
+
+size_t moe_route_workspace_size(const moe_dims* dims, int32_t T) {
+  if (dims == nullptr || T < 0) return 0;
+  return round_up((size_t)T * dims->n_experts * sizeof(float), 256);
+}
+
+moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float* router_w,
+                     const float* bias, const int32_t* token_ids, const int32_t* hash_table,
+                     int32_t vocab, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                     void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !router_w || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  const bool hashed = token_ids != nullptr || hash_table != nullptr;
+  if (hashed && (!token_ids || !hash_table || vocab <= 0)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(router_w, 16)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < moe_route_workspace_size(dims, T) || ws == nullptr) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int E = dims->n_experts, H = dims->hidden;
+  float* logits = static_cast<float*>(ws);
+  dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
+  route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
+  if ((st = launch_status()) != MOE_OK) return st;
+  route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
+      logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table,
+      vocab, topk_idx, topk_w);
+  return launch_status();
+}
+
+size_t moe_permute_workspace_size(int32_t T, int32_t K, int32_t E) {
+  (void)T; (void)K; (void)E;
+  return 0;
+}
+
+moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E, int32_t* offsets,
+                       int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  if (T < 0 || K <= 0 || E <= 0 || E > 1024 || K > 32) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)T * K > (1 << 22)) return MOE_ERR_UNSUPPORTED;
+  if (!offsets || (T > 0 && (!topk_idx || !perm || !inv))) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int smem = 32 * E * (int)sizeof(int32_t);
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * 4) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = true;
+  }
+  permute_kernel<<<1, kPermuteThreads, smem, s>>>(topk_idx, T * K, E, offsets, perm, inv);
+  return launch_status();
+}
+
+size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
+  if (dims == nullptr || T < 0) return 0;
+  return round_up((size_t)T * dims->top_k * dims->inter * sizeof(float), 256);
+}
+
+moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
+                           moe_mxfp4_proj up, moe_mxfp4_proj down, const int32_t* offsets,
+                           const int32_t* perm, float* y_perm, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !offsets || !perm || !y_perm) return MOE_ERR_INVALID_ARG;
+  const int H = dims->hidden, I = dims->inter;
+  if ((st = check_proj(gate, I, H)) != MOE_OK) return st;
+  if ((st = check_proj(up, I, H)) != MOE_OK) return st;
+  if ((st = check_proj(down, H, I)) != MOE_OK) return st;
+  if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
+  if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* h = static_cast<float*>(ws);
+
+  GemvArgs a{};
+  a.a = {gate.base, gate.expert_bytes, gate.rows, gate.cols};
+  a.b = {up.base, up.expert_bytes, up.rows, up.cols};
+  a.limit = dims->swiglu_limit;
+  a.xin = x;
+  a.xin_f32 = 0;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.K = dims->top_k;
+  a.E = dims->n_experts;
+  a.out = h;
+  a.out_ld = I;
+  if ((st = launch_gemv<kWMxfp4, 2, 4>(a, s)) != MOE_OK) return st;
+
+  GemvArgs d{};
+  d.a = {down.base, down.expert_bytes, down.rows, down.cols};
+  d.b = d.a;
+  d.limit = dims->swiglu_limit;
+  d.xin = h;
+  d.xin_f32 = 1;
+  d.offsets = offsets;
+  d.perm = nullptr;
+  d.K = dims->top_k;
+  d.E = dims->n_experts;
+  d.out = y_perm;
+  d.out_ld = H;
+  return launch_gemv<kWMxfp4, 1, 4>(d, s);
+}
+
+size_t shared_expert_workspace_size(const moe_dims* dims, int32_t T) {
+  if (dims == nullptr || T < 0) return 0;
+  return round_up((size_t)T * dims->inter * sizeof(float), 256);
+}
+
+moe_status shared_expert(const moe_dims* dims, const void* x, int32_t T, const void* wg,
+                         const void* wu, const void* wd, float* out, void* ws, size_t ws_bytes,
+                         void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !wg || !wu || !wd || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(wg, 16) || !aligned(wu, 16) || !aligned(wd, 16) || !aligned(out, 16))
+    return MOE_ERR_ALIGNMENT;
+  if (ws == nullptr || ws_bytes < shared_expert_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = dims->hidden, I = dims->inter;
+  float* h = static_cast<float*>(ws);
+  GemvArgs a{};
+  a.a = {static_cast<const uint8_t*>(wg), 0, I, H};
+  a.b = {static_cast<const uint8_t*>(wu), 0, I, H};
+  a.limit = dims->swiglu_limit;
+  a.xin = x;
+  a.xin_f32 = 0;
+  a.offsets = nullptr;
+  a.perm = nullptr;
+  a.K = 1;
+  a.E = 1;
+  a.n_single = T;
+  a.out = h;
+  a.out_ld = I;
+  if ((st = launch_gemv<kWBf16, 2, 2>(a, s)) != MOE_OK) return st;
+  GemvArgs d = a;
+  d.a = {static_cast<const uint8_t*>(wd), 0, H, I};
+  d.b = d.a;
+  d.xin = h;
+  d.xin_f32 = 1;
+  d.out = out;
+  d.out_ld = H;
+  return launch_gemv<kWBf16, 1, 2>(d, s);
+}
+
+moe_status moe_combine(const moe_dims* dims, int32_t T, const float* y_perm, const int32_t* inv,
+                       const float* topk_w, const float* shared_out, float* out_f32, void* out_bf16,
+                       void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y_perm || !inv || !topk_w || !out_f32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y_perm, 16) || !aligned(out_f32, 16) || (shared_out && !aligned(shared_out, 16)) ||
+      (out_bf16 && !aligned(out_bf16, 8)))
+    return MOE_ERR_ALIGNMENT;
+  const int H = dims->hidden;
+  dim3 grid((H / 4 + kCombineThreads - 1) / kCombineThreads, T);
+  combine_kernel<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      y_perm, inv, topk_w, shared_out, out_f32, static_cast<__nv_bfloat16*>(out_bf16), dims->top_k, H);
+  return launch_status();
+}
+
+}  // extern "C"

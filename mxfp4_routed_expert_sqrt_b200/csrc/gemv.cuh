@@ -29,10 +29,11 @@ namespace moe {
 
 enum { kWMxfp4 = 0, kWBf16 = 1 };
 
-constexpr int kGemvThreads = 128;
+constexpr int kGemvThreads = 512;
 constexpr int kGemvStages = 4;
 constexpr int kGemvStageTarget = 36 * 1024;  // bytes of weights per stage (approx.)
 constexpr int kGemvRedFloats = 2048;         // cross-segment reduction buffer
+constexpr int kGemvSmemBudget = 200 * 1024;  // dynamic shared memory for the stage ring
 
 struct GemvProj {
   const uint8_t* base;   // expert 0
@@ -51,6 +52,7 @@ struct GemvArgs {
   int E;
   int n_single;
   int rb;                  // rows per unit (multiple of rp, divides rows)
+  int n_stages;            // depth of the shared-memory ring, 1..kGemvStages
   float* out;              // fp32 [pos][out_ld], column = weight row
   int out_ld;
 };
@@ -89,7 +91,7 @@ __device__ __forceinline__ float dot_group_mxfp4(const uint32_t (&w)[16], const 
 }
 
 template <int WF, int P, int RBI, int NTP>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args) {
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs args) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kGemvStages];
   __shared__ int32_t s_active[1024];
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
   if (u_begin >= u_end) return;
 
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages; ++s) mbar_init(&full_bar[s], 1);
+    for (int s = 0; s < kGemvStages; ++s) mbar_init(&full_bar[s], 1);  // all slots; n_stages used
     fence_mbar_init();
   }
   __syncthreads();
@@ -164,26 +166,27 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
       }
     }
   };
+  const int NS = args.n_stages;
   if (tid == 0)
-    for (int k = 0; k < kGemvStages && u_begin + k < u_end; ++k) issue(u_begin + k, k);
+    for (int k = 0; k < NS && u_begin + k < u_end; ++k) issue(u_begin + k, k);
 
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(args.xin);
   const float* xf = static_cast<const float*>(args.xin);
 
   for (int u = u_begin; u < u_end; ++u) {
-    const int k = u - u_begin, s = k % kGemvStages;
+    const int k = u - u_begin, s = k % NS;
     const int e = s_active[u / units_per_expert];
     const int r0 = (u % units_per_expert) * rb;
     int pos0, n_tok;
     if (args.offsets != nullptr) { pos0 = args.offsets[e]; n_tok = args.offsets[e + 1] - pos0; }
     else { pos0 = 0; n_tok = args.n_single; }
     // all threads agree on the outcome of the (bounded) wait
-    if (!__syncthreads_and(mbar_wait(&full_bar[s], (k / kGemvStages) & 1))) {
+    if (!__syncthreads_and(mbar_wait(&full_bar[s], (k / NS) & 1))) {
       if (tid == 0) {
         set_error(kErrWaitGemv);
         // let every copy already issued land before the CTA's shared memory goes away
-        for (int k2 = k + 1; k2 < min(u_end - u_begin, k + kGemvStages); ++k2)
-          mbar_wait(&full_bar[k2 % kGemvStages], (k2 / kGemvStages) & 1);
+        for (int k2 = k + 1; k2 < min(u_end - u_begin, k + NS); ++k2)
+          mbar_wait(&full_bar[k2 % NS], (k2 / NS) & 1);
       }
       return;
     }
@@ -197,6 +200,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
 #pragma unroll
       for (int j = 0; j < NTP; ++j) {
         const bool ok = j0 + j < n_tok;
+        if (!ok) continue;
         int row = 0;
         if (ok) {
           const int pos = pos0 + j0 + j;
@@ -254,7 +258,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
               e2m1x8_to_f16x2(nb.w, t4); w[12] = t4[0]; w[13] = t4[1]; w[14] = t4[2]; w[15] = t4[3];
             }
 #pragma unroll
-            for (int j = 0; j < NTP; ++j) part[p][ri][j] = dot_group_mxfp4(w, xv[j]) * sc;
+            for (int j = 0; j < NTP; ++j)
+              part[p][ri][j] = (j0 + j < n_tok) ? dot_group_mxfp4(w, xv[j]) * sc : 0.f;
           } else {
             const uint4* wr = reinterpret_cast<const uint4*>(pst + (int64_t)r * cols * 2 + g * 64);
             float acc[NTP];
@@ -269,8 +274,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
                 const float wlo = __uint_as_float(vv[i] << 16), whi = __uint_as_float(vv[i] & 0xFFFF0000u);
 #pragma unroll
                 for (int j = 0; j < NTP; ++j) {
-                  acc[j] = fmaf(wlo, xs[WF == kWBf16 ? j : 0][8 * c + 2 * i], acc[j]);
-                  acc[j] = fmaf(whi, xs[WF == kWBf16 ? j : 0][8 * c + 2 * i + 1], acc[j]);
+                  if (j0 + j < n_tok) {
+                    acc[j] = fmaf(wlo, xs[WF == kWBf16 ? j : 0][8 * c + 2 * i], acc[j]);
+                    acc[j] = fmaf(whi, xs[WF == kWBf16 ? j : 0][8 * c + 2 * i + 1], acc[j]);
+                  }
                 }
               }
             }
@@ -287,9 +294,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
         for (int ri = 0; ri < RBI; ++ri)
 #pragma unroll
           for (int j = 0; j < NTP; ++j) {
-            float v = part[p][ri][j];
-            for (int o = seg >> 1; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            part[p][ri][j] = v;
+            if (j0 + j < n_tok) {
+              float v = part[p][ri][j];
+              for (int o = seg >> 1; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              part[p][ri][j] = v;
+            }
           }
       // one writer per segment: s_red[segment][p][ri][j]
       const int seg_id = tid / seg;
@@ -323,8 +332,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs args)
       __syncthreads();
     }
 
-    // stage s is free again: refill it with unit u + kGemvStages
-    if (tid == 0 && u + kGemvStages < u_end) issue(u + kGemvStages, s);
+    // stage s is free again: refill it with unit u + NS
+    if (tid == 0 && u + NS < u_end) issue(u + NS, s);
   }
 }
 

@@ -7,6 +7,8 @@
 #include "gemv.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "tc_expert.cuh"
+#include "decode_mma.cuh"
 
 using namespace moe;
 
@@ -29,6 +31,78 @@ moe_status launch_status() {
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 [rows][cols] viewed by TMA with a {64, 1} box and 128-byte swizzle
+// (the gather4 operand layout of the tensor-core expert kernel).
+bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                  CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+moe_status launch_tc(const CUtensorMap& map, const TcArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(tc_expert_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = true;
+  }
+  tc_expert_kernel<MODE><<<sm_count(), kTcThreads, kTcSmem, s>>>(map, a);
+  return launch_status();
+}
+
+// Token counts up to this use the decode path (weight streaming with
+// register decode and warp MMA fragments); above it the tcgen05 grouped GEMM.
+constexpr int kGemvMaxT = 64;
+
+template <int MODE>
+int dec_stage_bytes(int cols) {
+  using L = DecLayout<MODE>;
+  return ((L::kRows * (cols / 2 + 16) + L::kRows * (cols / 32)) + 127) / 128 * 128;
+}
+
+template <int MODE>
+moe_status launch_dec(const DecArgs& a, cudaStream_t s) {
+  const int smem = dec_stage_bytes<MODE>(a.cols) * kDecStages;
+  if (smem > 110 * 1024) return MOE_ERR_UNSUPPORTED;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(decode_mma_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(decode_mma_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = true;
+  }
+  decode_mma_kernel<MODE><<<2 * sm_count(), kDecThreads, smem, s>>>(a);
+  return launch_status();
 }
 
 moe_status check_dims(const moe_dims* d) {
@@ -57,14 +131,17 @@ moe_status launch_gemv_inst(const GemvArgs& a, cudaStream_t s) {
   auto kern = gemv_kernel<WF, P, RBI, NTP>;
   const int64_t row_bytes = gemv_row_bytes(WF, a.a.cols);
   const int64_t stage = ((int64_t)P * a.rb * row_bytes + 127) / 128 * 128;
-  const int smem = (int)(stage * kGemvStages);
+    GemvArgs a2 = a;
+  a2.n_stages = (int)((kGemvSmemBudget / stage) < kGemvStages ? (kGemvSmemBudget / stage) : kGemvStages);
+  if (a2.n_stages < 1) return MOE_ERR_UNSUPPORTED;
+  const int smem = (int)(stage * a2.n_stages);
   static bool configured = false;  // per instantiation; the attribute is per function
   if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured = true;
   }
-  kern<<<sm_count(), kGemvThreads, smem, s>>>(a);
+  kern<<<sm_count(), kGemvThreads, smem, s>>>(a2);
   return launch_status();
 }
 
@@ -176,7 +253,11 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  return round_up((size_t)T * dims->top_k * dims->inter * sizeof(float), 256);
+  // decode path: x in f16 [T][hidden] and h in f16 [T*top_k][inter];
+  // tensor-core path: h in f16 [T*top_k][inter]
+  const size_t h = round_up((size_t)T * dims->top_k * dims->inter * 2, 256);
+  if (T <= kGemvMaxT) return round_up((size_t)T * dims->hidden * 2, 256) + h;
+  return h;
 }
 
 moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
@@ -195,35 +276,66 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
   if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* h = static_cast<float*>(ws);
-
-  GemvArgs a{};
-  a.a = {gate.base, gate.expert_bytes, gate.rows, gate.cols};
-  a.b = {up.base, up.expert_bytes, up.rows, up.cols};
-  a.limit = dims->swiglu_limit;
-  a.xin = x;
-  a.xin_f32 = 0;
+  if (T > kGemvMaxT) {
+    if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
+    __half* hb = static_cast<__half*>(ws);
+    CUtensorMap xmap, hmap;
+    if (!make_row_map(&xmap, x, T, H) ||
+        !make_row_map(&hmap, hb, (int64_t)T * dims->top_k, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      return MOE_ERR_CUDA;
+    TcArgs g{};
+    g.w0 = gate.base;
+    g.w1 = up.base;
+    g.expert_bytes = gate.expert_bytes;
+    g.rows = I;
+    g.cols = H;
+    g.offsets = offsets;
+    g.perm = perm;
+    g.K = dims->top_k;
+    g.E = dims->n_experts;
+    g.out = hb;
+    g.limit = dims->swiglu_limit;
+    if ((st = launch_tc<0>(xmap, g, s)) != MOE_OK) return st;
+    TcArgs d = g;
+    d.w0 = down.base;
+    d.w1 = nullptr;
+    d.expert_bytes = down.expert_bytes;
+    d.rows = H;
+    d.cols = I;
+    d.out = y_perm;
+    return launch_tc<1>(hmap, d, s);
+  }
+  if (H % 128 || I % 128 || I % 32 || H / 2 % 16) return MOE_ERR_UNSUPPORTED;
+  __half* x16 = static_cast<__half*>(ws);
+  __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)T * H * 2, 256));
+  const int64_t n8 = (int64_t)T * H / 8;
+  bf16_to_f16_kernel<<<(int)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184), 256, 0, s>>>(
+      static_cast<const uint4*>(x), reinterpret_cast<uint4*>(x16), n8);
+  if ((st = launch_status()) != MOE_OK) return st;
+  DecArgs a{};
+  a.w0 = gate.base;
+  a.w1 = up.base;
+  a.expert_bytes = gate.expert_bytes;
+  a.rows = I;
+  a.cols = H;
+  a.xin = x16;
   a.offsets = offsets;
   a.perm = perm;
   a.K = dims->top_k;
   a.E = dims->n_experts;
-  a.out = h;
-  a.out_ld = I;
-  if ((st = launch_gemv<kWMxfp4, 2, 4>(a, s)) != MOE_OK) return st;
-
-  GemvArgs d{};
-  d.a = {down.base, down.expert_bytes, down.rows, down.cols};
-  d.b = d.a;
-  d.limit = dims->swiglu_limit;
-  d.xin = h;
-  d.xin_f32 = 1;
-  d.offsets = offsets;
+  a.out = h16;
+  a.limit = dims->swiglu_limit;
+  if ((st = launch_dec<0>(a, s)) != MOE_OK) return st;
+  DecArgs d = a;
+  d.w0 = down.base;
+  d.w1 = nullptr;
+  d.expert_bytes = down.expert_bytes;
+  d.rows = H;
+  d.cols = I;
+  d.xin = h16;
   d.perm = nullptr;
-  d.K = dims->top_k;
-  d.E = dims->n_experts;
   d.out = y_perm;
-  d.out_ld = H;
-  return launch_gemv<kWMxfp4, 1, 4>(d, s);
+  return launch_dec<1>(d, s);
 }
 
 size_t shared_expert_workspace_size(const moe_dims* dims, int32_t T) {

@@ -1,0 +1,466 @@
+// Grouped expert GEMM on the 5th-generation tensor cores (tcgen05), for the
+// prefill / many-token regime.
+//
+// Per unit = (expert e, token chunk of <= 128 grouped pairs, 128-row tile):
+//   MODE 0 (gate/up):  acc0 = Wg[rows] x^T, acc1 = Wu[rows] x^T over K = hidden,
+//                      bf16 operands (x as given, weights dequantised exactly to
+//                      bf16); epilogue h = silu(min(acc0, L)) * clamp(acc1, -L, L)
+//                      stored in f16 (|h| <= L^2; 11 mantissa bits, 8x finer
+//                      than bf16, which keeps the output inside the error bar)
+//   MODE 1 (down):     acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter, f16
+//                      operands, fp32 out.  Weights are dequantised exactly to
+//                      f16 as v * 2^(e - 127 - c_r), with c_r = max(0, e_max(row)
+//                      - 140) undone in the epilogue: exact whenever a row's
+//                      exponents span at most 36.
+// ("Model techniques map", row "SwiGLU feed-forward": the clamped SwiGLU;
+// "ElytronAI / DeepSeek-v4-Flash", Sizes/Layout: MXFP4 weights, expert xid at
+// base + xid * expert_bytes.)
+//
+// Swap-AB: the weight rows are the MMA's M = 128 dimension and the expert's
+// tokens its N dimension (a multiple of 16, <= 128), so a unit needs no token
+// padding beyond 16.
+//
+// Roles (448 threads, one CTA per SM, persistent over units):
+//   warps 0-3   epilogue: tcgen05.ld of the two accumulators (TMEM lane
+//               quadrant = warp), SwiGLU or copy, global stores;
+//   warps 4-11  dequant: thread = one weight row of one of the two tiles; per
+//               64-column k-block it loads 32 B of E2M1 codes and 2 E8M0
+//               bytes, converts them EXACTLY to bf16 (E2M1 -> f16 by cvt, f16
+//               bits -> bf16 bits by a shift, times 2^(e-15) in bf16) and writes
+//               the 64 values into TMEM with tcgen05.st: the MMA takes its A
+//               operand from TMEM, so the weight tiles never touch shared memory;
+//   warp 12     token producer: TMA tile::gather4 of the unit's activation rows
+//               (bf16, 128-byte swizzle) into a 4-stage shared-memory ring;
+//   warp 13     TMEM owner and MMA issuer (one thread): 2 x 4 tcgen05.mma
+//               (M=128, N=n16, K=16) per k-block, tcgen05.commit to free stages.
+// TMEM (512 columns): acc0 [0,128), acc1 [128,256), A stages [256, 512).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kTcThreads = 448;
+constexpr int kTcStages = 4;
+constexpr int kTcKB = 64;     // k per stage (one 128-byte swizzle atom of bf16)
+constexpr int kTcNMax = 128;  // tokens per unit
+constexpr int kTcBTile = kTcNMax * kTcKB * 2;  // 16 KB per stage
+constexpr int kTcTmemCols = 512;
+constexpr int kTcAccCols = 128;
+constexpr int kTcAStage = 64;  // TMEM columns per stage: 2 tiles x 32
+constexpr int kTcSmemUsed = kTcStages * kTcBTile + 1024 /*align*/ + 8192 /*tables*/;
+// requested dynamic shared memory: more than half an SM's, so one CTA per SM
+// (each CTA owns all 512 TMEM columns)
+constexpr int kTcSmem = 120 * 1024;
+static_assert(kTcSmemUsed <= kTcSmem, "tc_expert shared memory");
+
+// ---- tcgen05 / TMA primitives --------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]^T
+__device__ __forceinline__ void umma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+        "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Four rows (r0..r3), 64 bf16 columns from col, of a 2-D tensor map whose box
+// is {64, 1} with 128-byte swizzle, into 512 contiguous bytes of shared memory.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int col, int r0, int r1, int r2,
+                                            int r3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 B apart (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 (or f16) A and B, both K-major, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Largest E8M0 exponent of a row's scale bytes (n multiple of 4, 4-byte aligned).
+__device__ __forceinline__ uint32_t row_max_e8m0(const uint8_t* sc, int n) {
+  uint32_t m = 0;
+  for (int i = 0; i < n; i += 4) m = __vmaxu4(m, *reinterpret_cast<const uint32_t*>(sc + i));
+  m = __vmaxu4(m, m >> 16);
+  m = __vmaxu4(m, m >> 8);
+  return m & 0xFFu;
+}
+
+// f16x2 with 2^k in both halves, k in [-24, 15] (subnormal f16 below -14).
+__device__ __forceinline__ uint32_t pow2_f16x2(int k) {
+  const float f = __uint_as_float((uint32_t)(k + 127) << 23);
+  return f32x2_to_f16x2(f, f);
+}
+
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Byte of two E2M1 codes -> bf16x2 of (value * 2^-112), exact: the f16 from
+// cvt has its exponent in bits 10-14 and mantissa bit 9; shifted right by 3
+// they sit in the low bits of the bf16 exponent and mantissa fields, i.e. the
+// value scaled by 2^(15-127).  Zero stays zero; the sign bits are kept.
+__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2_pre(uint32_t byte) {
+  const uint32_t h = e2m1x2_to_f16x2(byte);
+  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
+}
+
+// bf16x2 with 2^(e-15) in both halves (the factor that turns the pre form
+// into value * 2^(e-127)); valid for e <= 142.
+__device__ __forceinline__ uint32_t e8m0_pre_factor(uint32_t e) {
+  const uint32_t b = (e + 112u) << 7;
+  return b | (b << 16);
+}
+
+struct TcArgs {
+  const uint8_t* w0;     // MODE 0: gate blobs; MODE 1: down blobs
+  const uint8_t* w1;     // MODE 0: up blobs
+  int64_t expert_bytes;
+  int rows, cols;        // of one projection
+  const int32_t* offsets;
+  const int32_t* perm;   // MODE 0: token of pos = perm[pos] / K
+  int K, E;
+  void* out;             // MODE 0: bf16 h [pos][rows]; MODE 1: fp32 y [pos][rows]
+  float limit;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t a_full[kTcStages], b_full[kTcStages], empty[kTcStages];
+  __shared__ __align__(8) uint64_t acc_full, acc_empty;
+  __shared__ uint32_t s_taddr;
+  __shared__ int32_t s_abort;
+  __shared__ int32_t s_rows[kTcNMax];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kTcStages * kTcBTile);  // [E + 1]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = args.E;
+  const int MT = MODE == 0 ? args.rows / 128 : args.rows / 256;  // row tiles per expert
+  const int nkb = args.cols / kTcKB;
+
+  // ---- unit table: units(e) = MT * ceil(n_e / 128), exclusive prefix -------
+  if (warp == 0) {
+    int run = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int c = 0;
+      if (e < E) {
+        const int n = args.offsets[e + 1] - args.offsets[e];
+        c = MT * ((n + kTcNMax - 1) / kTcNMax);
+      }
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < E) s_prefix[e] = run + incl - c;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_prefix[E] = run;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&a_full[s], 8);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 4);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(&s_taddr, kTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = s_taddr;
+  const int n_units = s_prefix[E];
+
+  // unit -> (expert, chunk, row tile)
+  auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {  // last e with s_prefix[e] <= u
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    const int local = u - s_prefix[e];
+    mt = local % MT;
+    const int chunk = local / MT;
+    const int start = args.offsets[e];
+    const int ne = args.offsets[e + 1] - start;
+    pos0 = start + chunk * kTcNMax;
+    n = min(kTcNMax, ne - chunk * kTcNMax);
+  };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int32_t*>(&s_abort) != 0; };
+  auto give_up = [&]() {
+    set_error(kErrWaitTc);
+    *reinterpret_cast<volatile int32_t*>(&s_abort) = 1;
+  };
+
+  if (warp >= 4 && warp < 12) {
+    // ------------------------------ dequant ----------------------------------
+    const int t = (warp - 4) >> 2, q = warp & 3, r = q * 32 + lane;
+    uint32_t it = 0;
+    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int R = MODE == 0 ? mt * 128 + r : mt * 256 + t * 128 + r;
+      const uint8_t* blob = (MODE == 0 && t == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes;
+      const uint8_t* nib = blob + (int64_t)R * (args.cols / 2);
+      const uint8_t* scl = blob + (int64_t)args.rows * (args.cols / 2) + (int64_t)R * (args.cols / 32);
+      // MODE 1: per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
+      const int crow = MODE == 1 ? max(0, (int)row_max_e8m0(scl, args.cols / 32) - 140) : 0;
+      uint4 c0 = __ldg(reinterpret_cast<const uint4*>(nib));
+      uint4 c1 = __ldg(reinterpret_cast<const uint4*>(nib) + 1);
+      uint32_t sc = *reinterpret_cast<const uint16_t*>(scl);
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        uint4 n0 = c0, n1 = c1;
+        uint32_t nsc = sc;
+        if (kb + 1 < nkb) {  // next k-block's codes and scales in flight during this one
+          n0 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32));
+          n1 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32) + 1);
+          nsc = *reinterpret_cast<const uint16_t*>(scl + (kb + 1) * 2);
+        }
+        const uint32_t e0 = sc & 0xFFu, e1 = sc >> 8;
+        uint32_t v[32];
+        const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        if (MODE == 0) {
+          uint32_t f0 = e8m0_pre_factor(min(e0, 142u)), f1 = e8m0_pre_factor(min(e1, 142u));
+          // exponents above 142 do not fit one bf16 factor: apply 2^127 then the rest
+          const bool any_big = __any_sync(0xffffffffu, e0 > 142u || e1 > 142u);
+          const uint32_t g0 = e8m0_pre_factor(e0 > 142u ? e0 - 127u : 15u);
+          const uint32_t g1 = e8m0_pre_factor(e1 > 142u ? e1 - 127u : 15u);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              v[4 * c + b] = hmul2_bf16(e2m1x2_to_bf16x2_pre((wds[c] >> (8 * b)) & 0xFFu), c < 4 ? f0 : f1);
+          }
+          if (any_big) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = hmul2_bf16(v[i], i < 16 ? g0 : g1);
+          }
+        } else {
+          const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
+          const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t hv[4];
+            e2m1x8_to_f16x2(wds[c], hv);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
+          }
+        }
+        const int s = it % kTcStages;
+        if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
+        tc_fence_after();
+        tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
+        c0 = n0; c1 = n1; sc = nsc;
+      }
+    }
+  } else if (warp == 12) {
+    // ------------------------------ token producer ---------------------------
+    uint32_t it = 0;
+    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      for (int j = lane; j < n16; j += 32) {
+        const int p = pos0 + min(j, n - 1);  // pad rows repeat the last token
+        s_rows[j] = MODE == 0 ? args.perm[p] / args.K : p;
+      }
+      __syncwarp();
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kTcStages;
+        if (lane == 0) {
+          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); }
+          else {
+            mbar_arrive_expect_tx(&b_full[s], (uint32_t)n16 * kTcKB * 2);
+            uint8_t* dst = smem + s * kTcBTile;
+            for (int j = 0; j < n16; j += 4)
+              tma_gather4(dst + j * 128, &bmap, kb * kTcKB, s_rows[j], s_rows[j + 1], s_rows[j + 2], s_rows[j + 3],
+                          &b_full[s]);
+          }
+        }
+        __syncwarp();
+        if (aborted()) break;
+      }
+      __syncwarp();
+    }
+  } else if (warp == 13) {
+    // ------------------------------ MMA issuer --------------------------------
+    uint32_t it = 0, un = 0;
+    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      const uint32_t idesc = MODE == 0 ? idesc_bf16_f32(128, n16) : idesc_f16_f32(128, n16);
+      if (lane == 0) {
+        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) give_up();
+        tc_fence_after();
+      }
+      __syncwarp();
+      for (int kb = 0; kb < nkb && !aborted(); ++kb, ++it) {
+        const int s = it % kTcStages;
+        if (lane == 0) {
+          const uint32_t ph = (it / kTcStages) & 1;
+          if (!mbar_wait(&a_full[s], ph) || !mbar_wait(&b_full[s], ph)) { give_up(); }
+          else {
+            tc_fence_after();
+            const uint32_t bsa = smem_u32(smem + s * kTcBTile);
+            const uint32_t a0 = tbase + kTcTmemCols / 2 + s * kTcAStage;
+#pragma unroll
+            for (int ks = 0; ks < kTcKB / 16; ++ks) {
+              const uint64_t bd = sdesc_sw128(bsa + ks * 32);
+              const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+              umma_tmem_a(tbase, a0 + ks * 8, bd, idesc, acc);
+              umma_tmem_a(tbase + kTcAccCols, a0 + 32 + ks * 8, bd, idesc, acc);
+            }
+            umma_commit(&empty[s]);
+            if (kb == nkb - 1) umma_commit(&acc_full);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    // ------------------------------ epilogue ----------------------------------
+    const int q = warp;  // TMEM lanes 32q..32q+31
+    const int r = q * 32 + lane;
+    uint32_t un = 0;
+    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      if (!mbar_wait(&acc_full, un & 1)) { give_up(); break; }
+      tc_fence_after();
+      const uint32_t lrow = (uint32_t)(q * 32) << 16;
+      // MODE 1: undo the dequant's per-row offset 2^c_r (rows mt*256 + r and + 128)
+      float s0 = 1.f, s1 = 1.f;
+      if (MODE == 1) {
+        const uint8_t* blob = args.w0 + (int64_t)e * args.expert_bytes + (int64_t)args.rows * (args.cols / 2);
+        const int cr0 = max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + r) * (args.cols / 32), args.cols / 32) - 140);
+        const int cr1 =
+            max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + 128 + r) * (args.cols / 32), args.cols / 32) - 140);
+        s0 = __uint_as_float((uint32_t)(cr0 + 127) << 23);
+        s1 = __uint_as_float((uint32_t)(cr1 + 127) << 23);
+      }
+      for (int c0 = 0; c0 < n; c0 += 16) {
+        uint32_t g[16], h[16];
+        tmem_ld16(tbase + lrow + c0, g);
+        tmem_ld16(tbase + lrow + kTcAccCols + c0, h);
+        tmem_ld_wait();
+        if (MODE == 0) {
+          __half* out = static_cast<__half*>(args.out);
+          const int col = mt * 128 + r;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n)
+              out[(int64_t)(pos0 + c0 + j) * args.rows + col] =
+                  __float2half_rn(silu_clamped_swiglu(__uint_as_float(g[j]), __uint_as_float(h[j]), args.limit));
+        } else {
+          float* out = static_cast<float*>(args.out);
+          const int col = mt * 256 + r;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n) {
+              out[(int64_t)(pos0 + c0 + j) * args.rows + col] = __uint_as_float(g[j]) * s0;
+              out[(int64_t)(pos0 + c0 + j) * args.rows + col + 128] = __uint_as_float(h[j]) * s1;
+            }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTcTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -154,8 +154,11 @@ def _expert_gemm(dc, T):
     return idx, perm.cpu().numpy()[:T * K], y[:T * K * H].view(T * K, H).cpu().numpy()
 
 
+# T <= 64 runs the decode path, larger T the tensor-core grouped GEMM
 EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64), ("tiny_T37", gen.TINY, 37, 74), ("v4_T1", gen.V4, 1, 6),
-                ("v4_T8", gen.V4, 8, 48), ("v4_T37", gen.V4, 37, 24), ("v4_T64", gen.V4, 64, 24)]
+                ("v4_T8", gen.V4, 8, 48), ("v4_T37", gen.V4, 37, 24), ("v4_T64", gen.V4, 64, 24),
+                ("tiny_T100_tc", gen.TINY, 100, 200), ("tiny_T1000_tc", gen.TINY, 1000, 120),
+                ("v4_T96_tc", gen.V4, 96, 24), ("v4_T300_tc", gen.V4, 300, 24)]
 
 
 @pytest.mark.parametrize("name,dims,T,nsample", EXPERT_CASES, ids=[c[0] for c in EXPERT_CASES])

@@ -118,6 +118,36 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
                      int32_t vocab, int32_t* topk_idx, float* topk_w, void* ws,
                      size_t ws_bytes, void* stream);
 
+/*
+ * moe_route_noalloc: the same routing as moe_route, for callers that cannot
+ * allocate device memory at all -- for example a serving runtime that hands
+ * every byte of the device to its own pool at start-up, or embedding code
+ * that must not call cudaMalloc/cudaFree on its hot path.  The pages describe
+ * no such interface; this entry point has no counterpart there.
+ *
+ * Instead of a caller workspace it uses one scratch array that the library
+ * keeps in device memory (a file-scope __device__ array of
+ * MOE_ROUTE_NOALLOC_MAX_LOGITS floats, 256 KiB, present on every device that
+ * loads libmoe.so until the process exits).  Limits and behaviour:
+ *  - T * n_experts must not exceed MOE_ROUTE_NOALLOC_MAX_LOGITS; larger calls
+ *    return MOE_ERR_UNSUPPORTED and enqueue nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.  A failed lookup returns MOE_ERR_CUDA.
+ *  - All calls share the one array: two calls whose kernels overlap on the
+ *    GPU (different streams without ordering) race on it and may return
+ *    each other's scores.  Order such calls on one stream.
+ *  - The array keeps the previous call's logits; every call overwrites the
+ *    T * n_experts entries it reads before reading them, so nothing has to
+ *    start at zero.
+ * Arguments and outputs are those of moe_route (no ws / ws_bytes).
+ * No device memory is allocated or freed by this call.
+ */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS 65536
+moe_status moe_route_noalloc(const moe_dims* dims, const void* x, int32_t T, const float* router_w,
+                             const float* bias, const int32_t* token_ids, const int32_t* hash_table,
+                             int32_t vocab, int32_t* topk_idx, float* topk_w, void* stream);
+
 /* --- grouping ----------------------------------------------------------- */
 
 size_t moe_permute_workspace_size(int32_t T, int32_t K, int32_t E);

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3
 
 # every symbol include/moe.h declares
 EXPORTS = ("moe_abi_version", "moe_status_string", "moe_device_error", "moe_route_workspace_size",
-           "moe_route", "moe_permute_workspace_size", "moe_permute",
+           "moe_route", "moe_route_noalloc", "moe_permute_workspace_size", "moe_permute",
            "moe_expert_gemm_workspace_size", "moe_expert_gemm", "shared_expert_workspace_size",
            "shared_expert", "moe_combine")
 
@@ -65,6 +65,8 @@ def lib():
         L.moe_route_workspace_size.argtypes = [dp, _i32]
         L.moe_route.restype = ctypes.c_int
         L.moe_route.argtypes = [dp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]
+        L.moe_route_noalloc.restype = ctypes.c_int
+        L.moe_route_noalloc.argtypes = [dp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
         L.moe_permute_workspace_size.restype = _sz
         L.moe_permute_workspace_size.argtypes = [_i32, _i32, _i32]
         L.moe_permute.restype = ctypes.c_int
@@ -140,6 +142,21 @@ def moe_route(dims, x, T, router_w, bias, token_ids, hash_table, vocab, topk_idx
     _check("moe_route", lib().moe_route(ctypes.byref(dims_of(dims)), _ptr(x), T, _ptr(router_w), _ptr(bias),
                                         _ptr(token_ids), _ptr(hash_table), vocab, _ptr(topk_idx),
                                         _ptr(topk_w), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+ROUTE_NOALLOC_MAX_LOGITS = 65536
+
+
+def moe_route_noalloc(dims, x, T, router_w, bias, token_ids, hash_table, vocab, topk_idx, topk_w, stream=None):
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory: the logits go to a scratch array the library keeps on each
+    device (T * n_experts <= ROUTE_NOALLOC_MAX_LOGITS).  Calls share that
+    array, so calls that may overlap on the GPU must be ordered on one
+    stream.  The first call on a device sets up the array's address and
+    should come before any stream capture."""
+    _check("moe_route_noalloc", lib().moe_route_noalloc(ctypes.byref(dims_of(dims)), _ptr(x), T, _ptr(router_w),
+                                                        _ptr(bias), _ptr(token_ids), _ptr(hash_table), vocab,
+                                                        _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
 
 
 def moe_permute_workspace_size(T, K, E) -> int:

@@ -1,6 +1,7 @@
 // libmoe.so: the C ABI declared in include/moe.h.  One translation unit: the
 // kernels live in the headers included below.
 #include <cstdio>
+#include <mutex>
 
 #include "combine.cuh"
 #include "common.cuh"
@@ -173,6 +174,35 @@ moe_status launch_gemv(GemvArgs a, cudaStream_t s) {
 
 }  // namespace
 
+// ---- routing without a caller workspace -------------------------------------
+// Scratch for moe_route_noalloc: the logits of one call, T * n_experts floats.
+// Lives in device memory on every device that loads the library.
+static __device__ __align__(256) float g_route_noalloc_logits[MOE_ROUTE_NOALLOC_MAX_LOGITS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device; looked up once
+// per device (the host-side symbol is not a device address).
+cudaError_t noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_noalloc_logits);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
 extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
@@ -224,6 +254,31 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
   route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
       logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table,
       vocab, topk_idx, topk_w);
+  return launch_status();
+}
+
+moe_status moe_route_noalloc(const moe_dims* dims, const void* x, int32_t T, const float* router_w,
+                             const float* bias, const int32_t* token_ids, const int32_t* hash_table,
+                             int32_t vocab, int32_t* topk_idx, float* topk_w, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !router_w || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)T * dims->n_experts > MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_UNSUPPORTED;
+  const bool hashed = token_ids != nullptr || hash_table != nullptr;
+  if (hashed && (!token_ids || !hash_table || vocab <= 0)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(router_w, 16)) return MOE_ERR_ALIGNMENT;
+  float* logits = nullptr;
+  if (noalloc_scratch(&logits) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int E = dims->n_experts, H = dims->hidden;
+  dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
+  route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
+  if ((st = launch_status()) != MOE_OK) return st;
+  route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
+      logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table, vocab,
+      topk_idx, topk_w);
   return launch_status();
 }
 

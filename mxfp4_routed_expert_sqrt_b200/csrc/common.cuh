@@ -15,7 +15,7 @@ namespace moe {
 // Device error codes written to g_error (first writer wins).
 enum : int32_t {
   kErrNone = 0,
-  kErrWaitGemv = 0x101,     // expert/shared GEMV gave up waiting for a bulk copy
+  kErrWaitDecode = 0x101,   // decode expert kernel gave up waiting for a bulk copy
   kErrBadExpert = 0x201,    // an expert id outside [0, E) reached moe_permute
   kErrWaitTc = 0x301,       // tensor-core kernel gave up waiting on an mbarrier
 };
@@ -72,17 +72,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // 1-D bulk copy global -> shared (async proxy), completion counted in bytes
-// on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Same, with an L2 evict-first hint: streamed expert weights are read once.
+// on `bar`, with an L2 evict-first hint (streamed expert weights are read
+// once).  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s_stream(void* smem_dst, const void* gmem_src,
                                                 uint32_t bytes, uint64_t* bar, uint64_t policy) {
   asm volatile(
@@ -96,11 +87,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-
-// E8M0 exponent byte -> fp32 scale 2^(e-127), exact (e = 0 is the subnormal 2^-127).
-__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
-  return e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);
 }
 
 // Two E2M1 codes (one byte, low nibble first) -> f16x2 (low half = low nibble).
@@ -136,36 +122,10 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
-}
-
-// acc (f32) += both halves of an f16x2 (mixed-precision adds: no f16 rounding).
-__device__ __forceinline__ float add_f16x2_to_f32(uint32_t h2, float acc) {
-  float r;
-  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n"
-      " add.rn.f32.f16 %0, lo, %2;\n add.rn.f32.f16 %0, hi, %0;\n}\n"
-      : "=f"(r)
-      : "r"(h2), "f"(acc));
-  return r;
-}
-
-// acc += a.lo*b.lo + a.hi*b.hi, with bf16 sources and fp32 products/sums.
-__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float acc) {
-  float r;
-  asm("{\n .reg .b16 alo, ahi, blo, bhi;\n mov.b32 {alo, ahi}, %1;\n mov.b32 {blo, bhi}, %2;\n"
-      " fma.rn.f32.bf16 %0, alo, blo, %3;\n fma.rn.f32.bf16 %0, ahi, bhi, %0;\n}\n"
-      : "=f"(r)
-      : "r"(a), "r"(b), "f"(acc));
-  return r;
 }
 
 __device__ __forceinline__ float silu_clamped_swiglu(float g, float u, float limit) {

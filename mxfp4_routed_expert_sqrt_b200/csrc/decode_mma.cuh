@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mma_kernel(const DecArg
     const int pos0 = args.offsets[e], n_tok = args.offsets[e + 1] - pos0;
     if (!__syncthreads_and(mbar_wait(&full_bar[s], (k / kDecStages) & 1))) {
       if (tid == 0) {
-        set_error(kErrWaitGemv);
+        set_error(kErrWaitDecode);
         for (int k2 = k + 1; k2 < min(u_end - u_begin, k + kDecStages); ++k2)
           mbar_wait(&full_bar[k2 % kDecStages], (k2 / kDecStages) & 1);
       }

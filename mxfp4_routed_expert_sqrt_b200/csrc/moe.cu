@@ -5,11 +5,11 @@
 
 #include "combine.cuh"
 #include "common.cuh"
-#include "gemv.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 #include "tc_expert.cuh"
 #include "decode_mma.cuh"
+#include "shared_decode.cuh"
 
 using namespace moe;
 
@@ -66,22 +66,31 @@ bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, int AF>
 moe_status launch_tc(const CUtensorMap& map, const TcArgs& a, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_expert_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
+    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
     configured = true;
   }
-  tc_expert_kernel<MODE><<<sm_count(), kTcThreads, kTcSmem, s>>>(map, a);
+  tc_expert_kernel<MODE, AF><<<sm_count(), kTcThreads, kTcSmem, s>>>(map, a);
   return launch_status();
+}
+
+// Router and shared expert run on the tensor cores above this token count
+// (and when their shapes fit the kernel's tiles).
+constexpr int kTcMinT = 65;
+
+bool tc_router_ok(const moe_dims* d, int T) { return T >= kTcMinT && d->n_experts % 256 == 0 && d->hidden % 64 == 0; }
+bool tc_shared_ok(const moe_dims* d, int T) {
+  return T >= kTcMinT && d->inter % 128 == 0 && d->hidden % 256 == 0 && d->hidden % 64 == 0 && d->inter % 64 == 0;
 }
 
 // Token counts up to this use the decode path (weight streaming with
 // register decode and warp MMA fragments); above it the tcgen05 grouped GEMM.
-constexpr int kGemvMaxT = 64;
+constexpr int kDecodeMaxT = 64;
 
 template <int MODE>
 int dec_stage_bytes(int cols) {
@@ -123,53 +132,6 @@ moe_status check_proj(const moe_mxfp4_proj& p, int rows, int cols) {
   if (p.expert_bytes != (int64_t)rows * cols / 2 + (int64_t)rows * cols / 32) return MOE_ERR_INVALID_ARG;
   if (!aligned(p.base, 32) || p.expert_bytes % 16) return MOE_ERR_ALIGNMENT;
   return MOE_OK;
-}
-
-// ---- GEMV launch ----------------------------------------------------------
-
-template <int WF, int P, int RBI, int NTP>
-moe_status launch_gemv_inst(const GemvArgs& a, cudaStream_t s) {
-  auto kern = gemv_kernel<WF, P, RBI, NTP>;
-  const int64_t row_bytes = gemv_row_bytes(WF, a.a.cols);
-  const int64_t stage = ((int64_t)P * a.rb * row_bytes + 127) / 128 * 128;
-    GemvArgs a2 = a;
-  a2.n_stages = (int)((kGemvSmemBudget / stage) < kGemvStages ? (kGemvSmemBudget / stage) : kGemvStages);
-  if (a2.n_stages < 1) return MOE_ERR_UNSUPPORTED;
-  const int smem = (int)(stage * a2.n_stages);
-  static bool configured = false;  // per instantiation; the attribute is per function
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured = true;
-  }
-  kern<<<sm_count(), kGemvThreads, smem, s>>>(a2);
-  return launch_status();
-}
-
-// Rows per unit: RBI * rp, with the largest RBI in {16, 8, 4, 2, 1} whose
-// stage fits the byte target and whose row block divides the rows, keeping
-// the scale block a multiple of 16 bytes.
-template <int WF, int P, int NTP>
-moe_status launch_gemv(GemvArgs a, cudaStream_t s) {
-  const int gpr = a.a.cols / 32, rp = kGemvThreads / gpr;
-  const int64_t row_bytes = gemv_row_bytes(WF, a.a.cols);
-  for (int rbi = 16; rbi >= 1; rbi >>= 1) {
-    const int rb = rbi * rp;
-    if (a.a.rows % rb) continue;
-    if (rbi > 1 && (int64_t)P * rb * row_bytes > kGemvStageTarget) continue;
-    if (WF == kWMxfp4 && ((int64_t)rb * (a.a.cols / 32)) % 16) continue;
-    const int seg = gpr < 32 ? gpr : 32;
-    if ((kGemvThreads / seg) * P * rbi * NTP > kGemvRedFloats) continue;
-    a.rb = rb;
-    switch (rbi) {
-      case 16: return launch_gemv_inst<WF, P, 16, NTP>(a, s);
-      case 8: return launch_gemv_inst<WF, P, 8, NTP>(a, s);
-      case 4: return launch_gemv_inst<WF, P, 4, NTP>(a, s);
-      case 2: return launch_gemv_inst<WF, P, 2, NTP>(a, s);
-      default: return launch_gemv_inst<WF, P, 1, NTP>(a, s);
-    }
-  }
-  return MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -229,7 +191,10 @@ int32_t moe_device_error(void) {
 
 size_t moe_route_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  return round_up((size_t)T * dims->n_experts * sizeof(float), 256);
+  size_t b = round_up((size_t)T * dims->n_experts * sizeof(float), 256);
+  // tensor-core router: the router weight split into bf16 hi | mid | lo
+  if (tc_router_ok(dims, T)) b += round_up((size_t)dims->n_experts * 3 * dims->hidden * 2, 256);
+  return b;
 }
 
 moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float* router_w,
@@ -248,9 +213,29 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int E = dims->n_experts, H = dims->hidden;
   float* logits = static_cast<float*>(ws);
-  dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
-  route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
-  if ((st = launch_status()) != MOE_OK) return st;
+  if (tc_router_ok(dims, T)) {
+    // logits = x . (hi + mid + lo) on the tensor cores: every product exact, fp32 sums
+    __nv_bfloat16* split = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) +
+                                                            round_up((size_t)T * E * sizeof(float), 256));
+    split3_bf16_kernel<<<2 * sm_count(), 256, 0, s>>>(router_w, split, E, H);
+    if ((st = launch_status()) != MOE_OK) return st;
+    CUtensorMap xmap;
+    if (!make_row_map(&xmap, x, T, H)) return MOE_ERR_CUDA;
+    TcArgs a{};
+    a.w0 = reinterpret_cast<const uint8_t*>(split);
+    a.rows = E;
+    a.a_cols = 3 * H;
+    a.k_total = 3 * H;
+    a.b_cols = H;
+    a.n_single = T;
+    a.n_chunk = 32;
+    a.out = logits;
+    if ((st = launch_tc<1, kABf16>(xmap, a, s)) != MOE_OK) return st;
+  } else {
+    dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
+    route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
+    if ((st = launch_status()) != MOE_OK) return st;
+  }
   route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
       logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table,
       vocab, topk_idx, topk_w);
@@ -311,7 +296,7 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   // decode path: x in f16 [T][hidden] and h in f16 [T*top_k][inter];
   // tensor-core path: h in f16 [T*top_k][inter]
   const size_t h = round_up((size_t)T * dims->top_k * dims->inter * 2, 256);
-  if (T <= kGemvMaxT) return round_up((size_t)T * dims->hidden * 2, 256) + h;
+  if (T <= kDecodeMaxT) return round_up((size_t)T * dims->hidden * 2, 256) + h;
   return h;
 }
 
@@ -331,7 +316,7 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
   if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (T > kGemvMaxT) {
+  if (T > kDecodeMaxT) {
     if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
     __half* hb = static_cast<__half*>(ws);
     CUtensorMap xmap, hmap;
@@ -343,22 +328,28 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
     g.w1 = up.base;
     g.expert_bytes = gate.expert_bytes;
     g.rows = I;
-    g.cols = H;
+    g.a_cols = H;
+    g.k_total = H;
+    g.b_cols = H;
     g.offsets = offsets;
     g.perm = perm;
     g.K = dims->top_k;
     g.E = dims->n_experts;
+    g.n_chunk = kTcNMax;
     g.out = hb;
     g.limit = dims->swiglu_limit;
-    if ((st = launch_tc<0>(xmap, g, s)) != MOE_OK) return st;
+    if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
     TcArgs d = g;
     d.w0 = down.base;
     d.w1 = nullptr;
     d.expert_bytes = down.expert_bytes;
     d.rows = H;
-    d.cols = I;
+    d.a_cols = I;
+    d.k_total = I;
+    d.b_cols = I;
+    d.perm = nullptr;
     d.out = y_perm;
-    return launch_tc<1>(hmap, d, s);
+    return launch_tc<1, kAMxfp4>(hmap, d, s);
   }
   if (H % 128 || I % 128 || I % 32 || H / 2 % 16) return MOE_ERR_UNSUPPORTED;
   __half* x16 = static_cast<__half*>(ws);
@@ -411,29 +402,59 @@ moe_status shared_expert(const moe_dims* dims, const void* x, int32_t T, const v
   if (ws == nullptr || ws_bytes < shared_expert_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden, I = dims->inter;
-  float* h = static_cast<float*>(ws);
-  GemvArgs a{};
-  a.a = {static_cast<const uint8_t*>(wg), 0, I, H};
-  a.b = {static_cast<const uint8_t*>(wu), 0, I, H};
-  a.limit = dims->swiglu_limit;
-  a.xin = x;
-  a.xin_f32 = 0;
-  a.offsets = nullptr;
-  a.perm = nullptr;
-  a.K = 1;
-  a.E = 1;
-  a.n_single = T;
-  a.out = h;
-  a.out_ld = I;
-  if ((st = launch_gemv<kWBf16, 2, 2>(a, s)) != MOE_OK) return st;
-  GemvArgs d = a;
-  d.a = {static_cast<const uint8_t*>(wd), 0, H, I};
-  d.b = d.a;
-  d.xin = h;
-  d.xin_f32 = 1;
+  if (tc_shared_ok(dims, T)) {
+    // h as an exact-to-16-bits bf16 pair [T][2I] (hi | lo): the down GEMM runs
+    // over K = 2I with the bf16 down weights repeated, so no operand is rounded
+    // below 16 significant bits
+    __nv_bfloat16* h2 = static_cast<__nv_bfloat16*>(ws);
+    CUtensorMap xmap, hmap;
+    if (!make_row_map(&xmap, x, T, H) || !make_row_map(&hmap, h2, T, 2 * I)) return MOE_ERR_CUDA;
+    TcArgs g{};
+    g.w0 = static_cast<const uint8_t*>(wg);
+    g.w1 = static_cast<const uint8_t*>(wu);
+    g.rows = I;
+    g.a_cols = H;
+    g.k_total = H;
+    g.b_cols = H;
+    g.n_single = T;
+    g.n_chunk = kTcNMax;
+    g.out = h2;
+    g.limit = dims->swiglu_limit;
+    if ((st = launch_tc<0, kABf16>(xmap, g, s)) != MOE_OK) return st;
+    TcArgs d = g;
+    d.w0 = static_cast<const uint8_t*>(wd);
+    d.w1 = nullptr;
+    d.rows = H;
+    d.a_cols = I;
+    d.k_total = 2 * I;
+    d.b_cols = 2 * I;
+    d.out = out;
+    return launch_tc<1, kABf16>(hmap, d, s);
+  }
+  if (H % 256 || I % 32 || 2 * I % 256 || T > 8 * kShMaxNt) return MOE_ERR_UNSUPPORTED;
+  __nv_bfloat16* h2 = static_cast<__nv_bfloat16*>(ws);
+  ShArgs g{};
+  g.w0 = static_cast<const __nv_bfloat16*>(wg);
+  g.w1 = static_cast<const __nv_bfloat16*>(wu);
+  g.rows = I;
+  g.a_cols = H;
+  g.k_total = H;
+  g.xin = static_cast<const __nv_bfloat16*>(x);
+  g.T = T;
+  g.out = h2;
+  g.limit = dims->swiglu_limit;
+  shared_decode_kernel<0><<<I / 8, kShThreads, 0, s>>>(g);
+  if ((st = launch_status()) != MOE_OK) return st;
+  ShArgs d = g;
+  d.w0 = static_cast<const __nv_bfloat16*>(wd);
+  d.w1 = nullptr;
+  d.rows = H;
+  d.a_cols = I;
+  d.k_total = 2 * I;
+  d.xin = h2;
   d.out = out;
-  d.out_ld = H;
-  return launch_gemv<kWBf16, 1, 2>(d, s);
+  shared_decode_kernel<1><<<H / 16, kShThreads, 0, s>>>(d);
+  return launch_status();
 }
 
 moe_status moe_combine(const moe_dims* dims, int32_t T, const float* y_perm, const int32_t* inv,

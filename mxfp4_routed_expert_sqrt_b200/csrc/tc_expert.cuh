@@ -180,19 +180,25 @@ __device__ __forceinline__ uint32_t e8m0_pre_factor(uint32_t e) {
   return b | (b << 16);
 }
 
+enum { kAMxfp4 = 0, kABf16 = 1 };
+
 struct TcArgs {
-  const uint8_t* w0;     // MODE 0: gate blobs; MODE 1: down blobs
-  const uint8_t* w1;     // MODE 0: up blobs
-  int64_t expert_bytes;
-  int rows, cols;        // of one projection
-  const int32_t* offsets;
-  const int32_t* perm;   // MODE 0: token of pos = perm[pos] / K
-  int K, E;
-  void* out;             // MODE 0: bf16 h [pos][rows]; MODE 1: fp32 y [pos][rows]
+  const uint8_t* w0;     // MODE 0: gate; MODE 1: down (or any bf16 [rows][a_cols] matrix)
+  const uint8_t* w1;     // MODE 0: up
+  int64_t expert_bytes;  // stride between experts (MXFP4); 0 for a single bf16 matrix
+  int rows;              // rows of one projection (the MMA's M extent)
+  int a_cols;            // columns of the weight matrix
+  int k_total;           // reduction length: a multiple of a_cols (A column = k mod a_cols)
+  int b_cols;            // columns of a B row (B column = k mod b_cols)
+  const int32_t* offsets;  // [E+1] grouped pairs; null: one group of n_single rows
+  const int32_t* perm;     // B row of pos = perm[pos] / K; null: B row = pos
+  int K, E, n_single;
+  int n_chunk;           // tokens per unit: multiple of 16, <= kTcNMax
+  void* out;             // see the epilogue
   float limit;
 };
 
-template <int MODE>
+template <int MODE, int AF>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -206,19 +212,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kTcStages * kTcBTile);  // [E + 1]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int E = args.E;
-  const int MT = MODE == 0 ? args.rows / 128 : args.rows / 256;  // row tiles per expert
-  const int nkb = args.cols / kTcKB;
+  const bool grouped = args.offsets != nullptr;
+  const int E = grouped ? args.E : 1;
+  const int MT = MODE == 0 ? args.rows / 128 : args.rows / 256;  // row tiles per group
+  const int nkb = args.k_total / kTcKB;
+  const int NC = args.n_chunk;
 
-  // ---- unit table: units(e) = MT * ceil(n_e / 128), exclusive prefix -------
+  // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
       int c = 0;
       if (e < E) {
-        const int n = args.offsets[e + 1] - args.offsets[e];
-        c = MT * ((n + kTcNMax - 1) / kTcNMax);
+        const int n = grouped ? args.offsets[e + 1] - args.offsets[e] : args.n_single;
+        c = MT * ((n + NC - 1) / NC);
       }
       int incl = c;
 #pragma unroll
@@ -252,7 +260,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tbase = s_taddr;
   const int n_units = s_prefix[E];
 
-  // unit -> (expert, chunk, row tile)
+  // unit -> (group, row tile, first position, tokens)
   auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {  // last e with s_prefix[e] <= u
@@ -263,10 +271,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int local = u - s_prefix[e];
     mt = local % MT;
     const int chunk = local / MT;
-    const int start = args.offsets[e];
-    const int ne = args.offsets[e + 1] - start;
-    pos0 = start + chunk * kTcNMax;
-    n = min(kTcNMax, ne - chunk * kTcNMax);
+    const int start = grouped ? args.offsets[e] : 0;
+    const int ne = grouped ? args.offsets[e + 1] - start : args.n_single;
+    pos0 = start + chunk * NC;
+    n = min(NC, ne - chunk * NC);
   };
   auto aborted = [&]() { return *reinterpret_cast<volatile int32_t*>(&s_abort) != 0; };
   auto give_up = [&]() {
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp >= 4 && warp < 12) {
-    // ------------------------------ dequant ----------------------------------
+    // ------------------------------ A producer ---------------------------------
     const int t = (warp - 4) >> 2, q = warp & 3, r = q * 32 + lane;
     uint32_t it = 0;
     for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
@@ -283,60 +291,90 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       decode_unit(u, e, mt, pos0, n);
       const int R = MODE == 0 ? mt * 128 + r : mt * 256 + t * 128 + r;
       const uint8_t* blob = (MODE == 0 && t == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes;
-      const uint8_t* nib = blob + (int64_t)R * (args.cols / 2);
-      const uint8_t* scl = blob + (int64_t)args.rows * (args.cols / 2) + (int64_t)R * (args.cols / 32);
-      // MODE 1: per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
-      const int crow = MODE == 1 ? max(0, (int)row_max_e8m0(scl, args.cols / 32) - 140) : 0;
-      uint4 c0 = __ldg(reinterpret_cast<const uint4*>(nib));
-      uint4 c1 = __ldg(reinterpret_cast<const uint4*>(nib) + 1);
-      uint32_t sc = *reinterpret_cast<const uint16_t*>(scl);
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        uint4 n0 = c0, n1 = c1;
-        uint32_t nsc = sc;
-        if (kb + 1 < nkb) {  // next k-block's codes and scales in flight during this one
-          n0 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32));
-          n1 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32) + 1);
-          nsc = *reinterpret_cast<const uint16_t*>(scl + (kb + 1) * 2);
+      if (AF == kAMxfp4) {
+        const uint8_t* nib = blob + (int64_t)R * (args.a_cols / 2);
+        const uint8_t* scl = blob + (int64_t)args.rows * (args.a_cols / 2) + (int64_t)R * (args.a_cols / 32);
+        // MODE 1: per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
+        const int crow = MODE == 1 ? max(0, (int)row_max_e8m0(scl, args.a_cols / 32) - 140) : 0;
+        uint4 c0 = __ldg(reinterpret_cast<const uint4*>(nib));
+        uint4 c1 = __ldg(reinterpret_cast<const uint4*>(nib) + 1);
+        uint32_t sc = *reinterpret_cast<const uint16_t*>(scl);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          uint4 n0 = c0, n1 = c1;
+          uint32_t nsc = sc;
+          if (kb + 1 < nkb) {  // next k-block's codes and scales in flight during this one
+            n0 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32));
+            n1 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32) + 1);
+            nsc = *reinterpret_cast<const uint16_t*>(scl + (kb + 1) * 2);
+          }
+          const uint32_t e0 = sc & 0xFFu, e1 = sc >> 8;
+          uint32_t v[32];
+          const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          if (MODE == 0) {
+            uint32_t f0 = e8m0_pre_factor(min(e0, 142u)), f1 = e8m0_pre_factor(min(e1, 142u));
+            // exponents above 142 do not fit one bf16 factor: apply 2^127 then the rest
+            const bool any_big = __any_sync(0xffffffffu, e0 > 142u || e1 > 142u);
+            const uint32_t g0 = e8m0_pre_factor(e0 > 142u ? e0 - 127u : 15u);
+            const uint32_t g1 = e8m0_pre_factor(e1 > 142u ? e1 - 127u : 15u);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+                v[4 * c + b] = hmul2_bf16(e2m1x2_to_bf16x2_pre((wds[c] >> (8 * b)) & 0xFFu), c < 4 ? f0 : f1);
+            }
+            if (any_big) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = hmul2_bf16(v[i], i < 16 ? g0 : g1);
+            }
+          } else {
+            const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
+            const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t hv[4];
+              e2m1x8_to_f16x2(wds[c], hv);
+#pragma unroll
+              for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
+            }
+          }
+          const int s = it % kTcStages;
+          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
+          tc_fence_after();
+          tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
+          c0 = n0; c1 = n1; sc = nsc;
         }
-        const uint32_t e0 = sc & 0xFFu, e1 = sc >> 8;
-        uint32_t v[32];
-        const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        if (MODE == 0) {
-          uint32_t f0 = e8m0_pre_factor(min(e0, 142u)), f1 = e8m0_pre_factor(min(e1, 142u));
-          // exponents above 142 do not fit one bf16 factor: apply 2^127 then the rest
-          const bool any_big = __any_sync(0xffffffffu, e0 > 142u || e1 > 142u);
-          const uint32_t g0 = e8m0_pre_factor(e0 > 142u ? e0 - 127u : 15u);
-          const uint32_t g1 = e8m0_pre_factor(e1 > 142u ? e1 - 127u : 15u);
+      } else {
+        // bf16 rows, copied as they are; column = k mod a_cols
+        const uint4* row = reinterpret_cast<const uint4*>(blob + (int64_t)R * args.a_cols * 2);
+        uint4 cur[8], nxt[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+        for (int i = 0; i < 8; ++i) cur[i] = __ldg(row + i);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          if (kb + 1 < nkb) {
+            const int c16 = (((kb + 1) * kTcKB) % args.a_cols) / 8;
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
-              v[4 * c + b] = hmul2_bf16(e2m1x2_to_bf16x2_pre((wds[c] >> (8 * b)) & 0xFFu), c < 4 ? f0 : f1);
+            for (int i = 0; i < 8; ++i) nxt[i] = __ldg(row + c16 + i);
           }
-          if (any_big) {
+          uint32_t v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = hmul2_bf16(v[i], i < 16 ? g0 : g1);
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] = cur[i].x; v[4 * i + 1] = cur[i].y; v[4 * i + 2] = cur[i].z; v[4 * i + 3] = cur[i].w;
           }
-        } else {
-          const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
-          const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
+          const int s = it % kTcStages;
+          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
+          tc_fence_after();
+          tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t hv[4];
-            e2m1x8_to_f16x2(wds[c], hv);
-#pragma unroll
-            for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
-          }
+          for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
         }
-        const int s = it % kTcStages;
-        if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
-        tc_fence_after();
-        tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[s]);
-        c0 = n0; c1 = n1; sc = nsc;
       }
     }
   } else if (warp == 12) {
@@ -348,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int n16 = (n + 15) & ~15;
       for (int j = lane; j < n16; j += 32) {
         const int p = pos0 + min(j, n - 1);  // pad rows repeat the last token
-        s_rows[j] = MODE == 0 ? args.perm[p] / args.K : p;
+        s_rows[j] = args.perm != nullptr ? args.perm[p] / args.K : p;
       }
       __syncwarp();
       for (int kb = 0; kb < nkb; ++kb, ++it) {
@@ -358,8 +396,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           else {
             mbar_arrive_expect_tx(&b_full[s], (uint32_t)n16 * kTcKB * 2);
             uint8_t* dst = smem + s * kTcBTile;
+            const int col = (kb * kTcKB) % args.b_cols;
             for (int j = 0; j < n16; j += 4)
-              tma_gather4(dst + j * 128, &bmap, kb * kTcKB, s_rows[j], s_rows[j + 1], s_rows[j + 2], s_rows[j + 3],
+              tma_gather4(dst + j * 128, &bmap, col, s_rows[j], s_rows[j + 1], s_rows[j + 2], s_rows[j + 3],
                           &b_full[s]);
           }
         }
@@ -375,7 +414,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
       const int n16 = (n + 15) & ~15;
-      const uint32_t idesc = MODE == 0 ? idesc_bf16_f32(128, n16) : idesc_f16_f32(128, n16);
+      // bf16 operands except the routed down projection, which runs in f16
+      const uint32_t idesc =
+          (AF == kAMxfp4 && MODE == 1) ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
       if (lane == 0) {
         if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) give_up();
         tc_fence_after();
@@ -406,6 +447,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------ epilogue ----------------------------------
+    // MODE 0, MXFP4: h = swiglu(gate, up) in f16 [pos][rows]
+    // MODE 0, bf16:  h as a bf16 pair, hi at [pos][col], lo = h - hi at [pos][rows + col]
+    // MODE 1:        fp32 [pos][rows], both row tiles
     const int q = warp;  // TMEM lanes 32q..32q+31
     const int r = q * 32 + lane;
     uint32_t un = 0;
@@ -415,13 +459,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&acc_full, un & 1)) { give_up(); break; }
       tc_fence_after();
       const uint32_t lrow = (uint32_t)(q * 32) << 16;
-      // MODE 1: undo the dequant's per-row offset 2^c_r (rows mt*256 + r and + 128)
+      // MXFP4 down: undo the A producer's per-row offset 2^c_r
       float s0 = 1.f, s1 = 1.f;
-      if (MODE == 1) {
-        const uint8_t* blob = args.w0 + (int64_t)e * args.expert_bytes + (int64_t)args.rows * (args.cols / 2);
-        const int cr0 = max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + r) * (args.cols / 32), args.cols / 32) - 140);
-        const int cr1 =
-            max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + 128 + r) * (args.cols / 32), args.cols / 32) - 140);
+      if (MODE == 1 && AF == kAMxfp4) {
+        const uint8_t* blob = args.w0 + (int64_t)e * args.expert_bytes + (int64_t)args.rows * (args.a_cols / 2);
+        const int cr0 =
+            max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + r) * (args.a_cols / 32), args.a_cols / 32) - 140);
+        const int cr1 = max(
+            0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + 128 + r) * (args.a_cols / 32), args.a_cols / 32) - 140);
         s0 = __uint_as_float((uint32_t)(cr0 + 127) << 23);
         s1 = __uint_as_float((uint32_t)(cr1 + 127) << 23);
       }
@@ -431,13 +476,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld16(tbase + lrow + kTcAccCols + c0, h);
         tmem_ld_wait();
         if (MODE == 0) {
-          __half* out = static_cast<__half*>(args.out);
           const int col = mt * 128 + r;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < n)
-              out[(int64_t)(pos0 + c0 + j) * args.rows + col] =
-                  __float2half_rn(silu_clamped_swiglu(__uint_as_float(g[j]), __uint_as_float(h[j]), args.limit));
+            if (c0 + j < n) {
+              const float hv = silu_clamped_swiglu(__uint_as_float(g[j]), __uint_as_float(h[j]), args.limit);
+              const int64_t o = (int64_t)(pos0 + c0 + j);
+              if (AF == kAMxfp4) {
+                static_cast<__half*>(args.out)[o * args.rows + col] = __float2half_rn(hv);
+              } else {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out) + o * 2 * args.rows;
+                out[col] = hi;
+                out[args.rows + col] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+              }
+            }
         } else {
           float* out = static_cast<float*>(args.out);
           const int col = mt * 256 + r;
@@ -460,6 +513,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tbase, kTcTmemCols);
+  }
+}
+
+// Router weight fp32 [n] -> three bf16 parts hi, mid, lo with w = hi + mid + lo
+// (to within 2^-24 |w|): hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid);
+// each difference is exact in fp32.  Laid out [rows][3 * cols]: hi | mid | lo.
+__global__ void split3_bf16_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ out, int rows,
+                                   int cols) {
+  const int64_t n = (int64_t)rows * cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t rr = i / cols, c = i % cols;
+    const float v = w[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __nv_bfloat16* o = out + rr * 3 * cols;
+    o[c] = hi;
+    o[cols + c] = mid;
+    o[2 * cols + c] = lo;
   }
 }
 

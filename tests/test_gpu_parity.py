@@ -92,8 +92,10 @@ ROUTE_CASES = [
     ("v4_T1", gen.V4, 1, None, False),
     ("v4_T64", gen.V4, 64, None, False),
     ("v4_T64_bias", gen.V4, 64, "zipf", False),
-    ("v4_T300", gen.V4, 300, None, False),
+    ("v4_T300", gen.V4, 300, None, False),          # T > 64: tensor-core logits
+    ("v4_T1000_bias", gen.V4, 1000, "zipf", False),
     ("v4_hash_T64", gen.V4, 64, None, True),
+    ("v4_hash_T500", gen.V4, 500, None, True),
 ]
 
 
@@ -183,7 +185,8 @@ def test_expert_gemm_parity(name, dims, T, nsample):
     assert mx <= MAX_TOL and mean <= MEAN_TOL, f"{name}: max {mx:.2e} mean {mean:.2e}"
 
 
-@pytest.mark.parametrize("dims,T", [(gen.TINY, 8), (gen.V4, 1), (gen.V4, 8), (gen.V4, 64)])
+@pytest.mark.parametrize("dims,T", [(gen.TINY, 8), (gen.TINY, 100), (gen.V4, 1), (gen.V4, 8), (gen.V4, 64),
+                                    (gen.V4, 65), (gen.V4, 300), (gen.V4, 4096)])
 def test_shared_expert_parity(dims, T):
     c = make_case(dims, T)
     dc = DeviceCase(c, DEV)
@@ -226,7 +229,15 @@ def test_combine_parity(T, K, H, with_shared, with_bf16):
 
 # ---- the whole layer -------------------------------------------------------------------
 
+def _zipf_bias():
+    import json
+    import os
+    k = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "zipf_kappa.json")))["kappa"]
+    return gen.zipf_bias(0, gen.V4.n_experts, k)
+
+
 LAYER_CASES = [("tiny_T8", gen.TINY, 8, None, False, 8), ("tiny_T1", gen.TINY, 1, None, False, 1),
+               ("v4_zipf_T32_layer0", gen.V4, 32, "zipf", False, 8),
                ("v4_decode_T1", gen.V4, 1, None, False, 1), ("v4_decode_T8", gen.V4, 8, None, False, 8),
                ("v4_decode_T32", gen.V4, 32, None, False, 8), ("v4_decode_T64", gen.V4, 64, None, False, 8),
                ("v4_hash_T2048", gen.V4, 2048, None, True, 6), ("v4_prefill_T4096", gen.V4, 4096, None, False, 6)]
@@ -234,7 +245,7 @@ LAYER_CASES = [("tiny_T8", gen.TINY, 8, None, False, 8), ("tiny_T1", gen.TINY, 1
 
 @pytest.mark.parametrize("name,dims,T,bias,hashed,nsample", LAYER_CASES, ids=[c[0] for c in LAYER_CASES])
 def test_layer_parity(name, dims, T, bias, hashed, nsample):
-    c = make_case(dims, T, hashed=hashed)
+    c = make_case(dims, T, hashed=hashed, bias=_zipf_bias() if bias == "zipf" else None)
     dc = DeviceCase(c, DEV)
     layer = m.MoeLayer(dims, T, DEV)
     out = _f32(T * dims.hidden)

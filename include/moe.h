@@ -172,15 +172,20 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  * All routed experts for the grouped pairs:
  *   y_perm[pos] = Wd_e (silu(min(Wg_e x_t, L)) * clamp(Wu_e x_t, -L, L))
  * for pos in [offsets[e], offsets[e+1]), p = perm[pos], t = p / top_k.
- *  x        bf16 [T][hidden], 16-byte aligned.
+ *  x        bf16 [T][hidden], 16-byte aligned; converted to f16 on the way
+ *           in, so |x| must stay below 65504 (values under 2^-14 keep f16
+ *           subnormal precision).
  *  gate, up MXFP4 [inter][hidden]; down MXFP4 [hidden][inter] (see
- *           moe_mxfp4_proj).  Weights are dequantised exactly; products and
- *           sums are fp32.
+ *           moe_mxfp4_proj).  Every weight is dequantised exactly (to f16, up
+ *           to a power of two per row undone in fp32) as long as the E8M0
+ *           exponents of one weight row span at most 36 octaves; products are
+ *           exact and sums fp32 on the tensor cores.  h between the two GEMMs
+ *           is f16.
  *  offsets, perm  as written by moe_permute.
  *  y_perm   fp32 [T*top_k][hidden] out.
  *  ws       device workspace of moe_expert_gemm_workspace_size() bytes.
- * The path (CUDA-core GEMV for small T, tensor-core grouped GEMM otherwise)
- * is chosen from T alone, never from device-side counts.
+ * One grouped tcgen05 GEMM pair for every T; the number of units follows the
+ * device-side counts, the launch does not depend on them.
  */
 moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
                            moe_mxfp4_proj up, moe_mxfp4_proj down, const int32_t* offsets,

@@ -8,7 +8,6 @@
 #include "permute.cuh"
 #include "route.cuh"
 #include "tc_expert.cuh"
-#include "decode_mma.cuh"
 #include "shared_decode.cuh"
 
 using namespace moe;
@@ -88,32 +87,9 @@ bool tc_shared_ok(const moe_dims* d, int T) {
   return T >= kTcMinT && d->inter % 128 == 0 && d->hidden % 256 == 0 && d->hidden % 64 == 0 && d->inter % 64 == 0;
 }
 
-// Token counts up to this use the decode path (weight streaming with
-// register decode and warp MMA fragments); above it the tcgen05 grouped GEMM.
-constexpr int kDecodeMaxT = 64;
+}  // namespace
 
-template <int MODE>
-int dec_stage_bytes(int cols) {
-  using L = DecLayout<MODE>;
-  return ((L::kRows * (cols / 2 + 16) + L::kRows * (cols / 32)) + 127) / 128 * 128;
-}
-
-template <int MODE>
-moe_status launch_dec(const DecArgs& a, cudaStream_t s) {
-  const int smem = dec_stage_bytes<MODE>(a.cols) * kDecStages;
-  if (smem > 110 * 1024) return MOE_ERR_UNSUPPORTED;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(decode_mma_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(decode_mma_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-            cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured = true;
-  }
-  decode_mma_kernel<MODE><<<2 * sm_count(), kDecThreads, smem, s>>>(a);
-  return launch_status();
-}
+namespace {
 
 moe_status check_dims(const moe_dims* d) {
   if (d == nullptr) return MOE_ERR_INVALID_ARG;
@@ -293,11 +269,8 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  // decode path: x in f16 [T][hidden] and h in f16 [T*top_k][inter];
-  // tensor-core path: h in f16 [T*top_k][inter]
-  const size_t h = round_up((size_t)T * dims->top_k * dims->inter * 2, 256);
-  if (T <= kDecodeMaxT) return round_up((size_t)T * dims->hidden * 2, 256) + h;
-  return h;
+  // x in f16 [T][hidden], then h in f16 [T*top_k][inter]
+  return round_up((size_t)T * dims->hidden * 2, 256) + round_up((size_t)T * dims->top_k * dims->inter * 2, 256);
 }
 
 moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
@@ -316,72 +289,44 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
   if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (T > kDecodeMaxT) {
-    if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
-    __half* hb = static_cast<__half*>(ws);
-    CUtensorMap xmap, hmap;
-    if (!make_row_map(&xmap, x, T, H) ||
-        !make_row_map(&hmap, hb, (int64_t)T * dims->top_k, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
-      return MOE_ERR_CUDA;
-    TcArgs g{};
-    g.w0 = gate.base;
-    g.w1 = up.base;
-    g.expert_bytes = gate.expert_bytes;
-    g.rows = I;
-    g.a_cols = H;
-    g.k_total = H;
-    g.b_cols = H;
-    g.offsets = offsets;
-    g.perm = perm;
-    g.K = dims->top_k;
-    g.E = dims->n_experts;
-    g.n_chunk = kTcNMax;
-    g.out = hb;
-    g.limit = dims->swiglu_limit;
-    if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
-    TcArgs d = g;
-    d.w0 = down.base;
-    d.w1 = nullptr;
-    d.expert_bytes = down.expert_bytes;
-    d.rows = H;
-    d.a_cols = I;
-    d.k_total = I;
-    d.b_cols = I;
-    d.perm = nullptr;
-    d.out = y_perm;
-    return launch_tc<1, kAMxfp4>(hmap, d, s);
-  }
-  if (H % 128 || I % 128 || I % 32 || H / 2 % 16) return MOE_ERR_UNSUPPORTED;
+  if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
   __half* x16 = static_cast<__half*>(ws);
   __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)T * H * 2, 256));
   const int64_t n8 = (int64_t)T * H / 8;
   bf16_to_f16_kernel<<<(int)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184), 256, 0, s>>>(
       static_cast<const uint4*>(x), reinterpret_cast<uint4*>(x16), n8);
   if ((st = launch_status()) != MOE_OK) return st;
-  DecArgs a{};
-  a.w0 = gate.base;
-  a.w1 = up.base;
-  a.expert_bytes = gate.expert_bytes;
-  a.rows = I;
-  a.cols = H;
-  a.xin = x16;
-  a.offsets = offsets;
-  a.perm = perm;
-  a.K = dims->top_k;
-  a.E = dims->n_experts;
-  a.out = h16;
-  a.limit = dims->swiglu_limit;
-  if ((st = launch_dec<0>(a, s)) != MOE_OK) return st;
-  DecArgs d = a;
+  CUtensorMap xmap, hmap;
+  if (!make_row_map(&xmap, x16, T, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_row_map(&hmap, h16, (int64_t)T * dims->top_k, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MOE_ERR_CUDA;
+  TcArgs g{};
+  g.w0 = gate.base;
+  g.w1 = up.base;
+  g.expert_bytes = gate.expert_bytes;
+  g.rows = I;
+  g.a_cols = H;
+  g.k_total = H;
+  g.b_cols = H;
+  g.offsets = offsets;
+  g.perm = perm;
+  g.K = dims->top_k;
+  g.E = dims->n_experts;
+  g.n_chunk = kTcNMax;
+  g.out = h16;
+  g.limit = dims->swiglu_limit;
+  if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
+  TcArgs d = g;
   d.w0 = down.base;
   d.w1 = nullptr;
   d.expert_bytes = down.expert_bytes;
   d.rows = H;
-  d.cols = I;
-  d.xin = h16;
+  d.a_cols = I;
+  d.k_total = I;
+  d.b_cols = I;
   d.perm = nullptr;
   d.out = y_perm;
-  return launch_dec<1>(d, s);
+  return launch_tc<1, kAMxfp4>(hmap, d, s);
 }
 
 size_t shared_expert_workspace_size(const moe_dims* dims, int32_t T) {

@@ -6,8 +6,8 @@
 // MODE 1: 16 down rows); its 8 warps split K.  Lanes load their m16n8k16
 // fragments of weights and activations straight from global memory (16 bytes
 // per lane per 32-column group, coalesced per row), bf16 x bf16 products are
-// exact and accumulate in fp32 inside the MMA.  The k-to-lane assignment is
-// the one of decode_mma.cuh: lane (g, t) owns columns 32G + 8t + [0, 8).
+// exact and accumulate in fp32 inside the MMA.  The k-to-lane assignment:
+// lane (g, t) owns columns 32G + 8t + [0, 8) of every 32-column group.
 //
 // MODE 0 writes h as a bf16 pair, hi = bf16(h) at [t][row] and lo = bf16(h -
 // hi) at [t][I + row]; MODE 1 runs over K = 2I with the down weights repeated

@@ -2,16 +2,17 @@
 // prefill / many-token regime.
 //
 // Per unit = (expert e, token chunk of <= 128 grouped pairs, 128-row tile):
-//   MODE 0 (gate/up):  acc0 = Wg[rows] x^T, acc1 = Wu[rows] x^T over K = hidden,
-//                      bf16 operands (x as given, weights dequantised exactly to
-//                      bf16); epilogue h = silu(min(acc0, L)) * clamp(acc1, -L, L)
-//                      stored in f16 (|h| <= L^2; 11 mantissa bits, 8x finer
-//                      than bf16, which keeps the output inside the error bar)
-//   MODE 1 (down):     acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter, f16
-//                      operands, fp32 out.  Weights are dequantised exactly to
-//                      f16 as v * 2^(e - 127 - c_r), with c_r = max(0, e_max(row)
-//                      - 140) undone in the epilogue: exact whenever a row's
-//                      exponents span at most 36.
+//   MODE 0 (gate/up):  acc0 = Wg[rows] x^T, acc1 = Wu[rows] x^T over K = hidden;
+//                      epilogue h = silu(min(acc0, L)) * clamp(acc1, -L, L),
+//                      stored in f16 (|h| <= L^2; 11 mantissa bits)
+//   MODE 1 (down):     acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter, fp32 out
+// MXFP4 operands run as f16 x f16 MMAs (fp32 accumulation): activations come
+// in f16 and each weight is dequantised exactly to f16 as v * 2^(e - 127 -
+// c_r), c_r = max(0, e_max(row) - 140), with 2^c_r applied to the fp32
+// accumulator row in the epilogue.  That is exact whenever a row's E8M0
+// exponents span at most 36 octaves, and costs two instructions per pair of
+// codes (cvt + multiply), which keeps the tensor cores, not the dequant, the
+// limit.  bf16 weights (shared expert, router) are copied as they are.
 // ("Model techniques map", row "SwiGLU feed-forward": the clamped SwiGLU;
 // "ElytronAI / DeepSeek-v4-Flash", Sizes/Layout: MXFP4 weights, expert xid at
 // base + xid * expert_bytes.)
@@ -23,12 +24,12 @@
 // Roles (448 threads, one CTA per SM, persistent over units):
 //   warps 0-3   epilogue: tcgen05.ld of the two accumulators (TMEM lane
 //               quadrant = warp), SwiGLU or copy, global stores;
-//   warps 4-11  dequant: thread = one weight row of one of the two tiles; per
-//               64-column k-block it loads 32 B of E2M1 codes and 2 E8M0
-//               bytes, converts them EXACTLY to bf16 (E2M1 -> f16 by cvt, f16
-//               bits -> bf16 bits by a shift, times 2^(e-15) in bf16) and writes
-//               the 64 values into TMEM with tcgen05.st: the MMA takes its A
-//               operand from TMEM, so the weight tiles never touch shared memory;
+//   warps 4-11  A producer: thread = one weight row of one of the two tiles;
+//               its raw k-blocks arrive through a private cp.async ring; per
+//               64-column k-block it converts the 32 code bytes exactly (see
+//               above) and writes the 64 values into TMEM with tcgen05.st: the
+//               MMA takes its A operand from TMEM, so the weight tiles never
+//               touch shared memory;
 //   warp 12     token producer: TMA tile::gather4 of the unit's activation rows
 //               (bf16, 128-byte swizzle) into a 4-stage shared-memory ring;
 //   warp 13     TMEM owner and MMA issuer (one thread): 2 x 4 tcgen05.mma
@@ -50,11 +51,33 @@ constexpr int kTcBTile = kTcNMax * kTcKB * 2;  // 16 KB per stage
 constexpr int kTcTmemCols = 512;
 constexpr int kTcAccCols = 128;
 constexpr int kTcAStage = 64;  // TMEM columns per stage: 2 tiles x 32
-constexpr int kTcSmemUsed = kTcStages * kTcBTile + 1024 /*align*/ + 8192 /*tables*/;
+// Raw A staging: every A-producer thread copies its own weight row's next
+// k-blocks with cp.async into a private ring, kRawStagesMx deep for MXFP4
+// (32 code bytes per k-block; the row's whole E8M0 row is fetched once per
+// unit) and kRawStagesBf deep for bf16 rows (128 bytes per k-block).  Code
+// planes are [stage][16-byte chunk][thread], so a warp's 16-byte reads are
+// contiguous.
+constexpr int kTcAThreads = 256;
+constexpr int kRawStagesMx = 6;
+constexpr int kRawStagesBf = 3;
+constexpr int kScaleRowMax = 128;  // E8M0 bytes per weight row held per producer thread (cols <= 4096)
+constexpr int kRawMxBytes = kRawStagesMx * 2 * kTcAThreads * 16 + kTcAThreads * kScaleRowMax;  // 80 KB
+constexpr int kRawBfBytes = kRawStagesBf * 8 * kTcAThreads * 16;                          // 96 KB
+constexpr int kRawBytes = kRawMxBytes > kRawBfBytes ? kRawMxBytes : kRawBfBytes;
+constexpr int kTcSmemUsed = kTcStages * kTcBTile + kRawBytes + 1024 /*align*/ + 8192 /*tables*/;
 // requested dynamic shared memory: more than half an SM's, so one CTA per SM
 // (each CTA owns all 512 TMEM columns)
-constexpr int kTcSmem = 120 * 1024;
-static_assert(kTcSmemUsed <= kTcSmem, "tc_expert shared memory");
+constexpr int kTcSmem = kTcSmemUsed;
+static_assert(kTcSmem > 114 * 1024 && kTcSmem <= 227 * 1024, "tc_expert shared memory");
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ---- tcgen05 / TMA primitives --------------------------------------------------
 
@@ -143,15 +166,6 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Largest E8M0 exponent of a row's scale bytes (n multiple of 4, 4-byte aligned).
-__device__ __forceinline__ uint32_t row_max_e8m0(const uint8_t* sc, int n) {
-  uint32_t m = 0;
-  for (int i = 0; i < n; i += 4) m = __vmaxu4(m, *reinterpret_cast<const uint32_t*>(sc + i));
-  m = __vmaxu4(m, m >> 16);
-  m = __vmaxu4(m, m >> 8);
-  return m & 0xFFu;
-}
-
 // f16x2 with 2^k in both halves, k in [-24, 15] (subnormal f16 below -14).
 __device__ __forceinline__ uint32_t pow2_f16x2(int k) {
   const float f = __uint_as_float((uint32_t)(k + 127) << 23);
@@ -162,22 +176,6 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
-}
-
-// Byte of two E2M1 codes -> bf16x2 of (value * 2^-112), exact: the f16 from
-// cvt has its exponent in bits 10-14 and mantissa bit 9; shifted right by 3
-// they sit in the low bits of the bf16 exponent and mantissa fields, i.e. the
-// value scaled by 2^(15-127).  Zero stays zero; the sign bits are kept.
-__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2_pre(uint32_t byte) {
-  const uint32_t h = e2m1x2_to_f16x2(byte);
-  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
-}
-
-// bf16x2 with 2^(e-15) in both halves (the factor that turns the pre form
-// into value * 2^(e-127)); valid for e <= 142.
-__device__ __forceinline__ uint32_t e8m0_pre_factor(uint32_t e) {
-  const uint32_t b = (e + 112u) << 7;
-  return b | (b << 16);
 }
 
 enum { kAMxfp4 = 0, kABf16 = 1 };
@@ -207,9 +205,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint32_t s_taddr;
   __shared__ int32_t s_abort;
   __shared__ int32_t s_rows[kTcNMax];
+  __shared__ int16_t s_crow[4][2][128];  // per-row f16 offsets c_r, ring over units
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kTcStages * kTcBTile);  // [E + 1]
+  uint8_t* s_raw = smem + kTcStages * kTcBTile;                                    // raw A ring
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(s_raw + kRawBytes);               // [E + 1]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool grouped = args.offsets != nullptr;
@@ -285,57 +285,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp >= 4 && warp < 12) {
     // ------------------------------ A producer ---------------------------------
     const int t = (warp - 4) >> 2, q = warp & 3, r = q * 32 + lane;
-    uint32_t it = 0;
-    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+    uint32_t it = 0, un_a = 0;
+    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un_a) {
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
       const int R = MODE == 0 ? mt * 128 + r : mt * 256 + t * 128 + r;
       const uint8_t* blob = (MODE == 0 && t == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes;
+      const int tslot = (warp - 4) * 32 + lane;
       if (AF == kAMxfp4) {
         const uint8_t* nib = blob + (int64_t)R * (args.a_cols / 2);
-        const uint8_t* scl = blob + (int64_t)args.rows * (args.a_cols / 2) + (int64_t)R * (args.a_cols / 32);
-        // MODE 1: per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
-        const int crow = MODE == 1 ? max(0, (int)row_max_e8m0(scl, args.a_cols / 32) - 140) : 0;
-        uint4 c0 = __ldg(reinterpret_cast<const uint4*>(nib));
-        uint4 c1 = __ldg(reinterpret_cast<const uint4*>(nib) + 1);
-        uint32_t sc = *reinterpret_cast<const uint16_t*>(scl);
+        const int sr = args.a_cols / 32;  // scale bytes per row (multiple of 4, <= kScaleRowMax)
+        const uint8_t* scl = blob + (int64_t)args.rows * (args.a_cols / 2) + (int64_t)R * sr;
+        uint8_t* my_sc = s_raw + kRawStagesMx * 2 * kTcAThreads * 16 + tslot * kScaleRowMax;
+        auto nib_at = [&](int st, int h) { return s_raw + ((st * 2 + h) * kTcAThreads + tslot) * 16; };
+        auto issue = [&](int kb2) {
+          cp_async16(nib_at(kb2 % kRawStagesMx, 0), nib + kb2 * 32);
+          cp_async16(nib_at(kb2 % kRawStagesMx, 1), nib + kb2 * 32 + 16);
+        };
+        // the row's E8M0 bytes in one go (first group), then the ring prologue
+        if (sr % 16 == 0) {
+          for (int i = 0; i < sr; i += 16) cp_async16(my_sc + i, scl + i);
+        } else {
+          for (int i = 0; i < sr; i += 4)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(my_sc + i)), "l"(scl + i)
+                         : "memory");
+        }
+        cp_async_commit();
+#pragma unroll
+        for (int p = 0; p < kRawStagesMx - 1; ++p) {
+          if (p < nkb) issue(p);
+          cp_async_commit();
+        }
+        cp_async_wait<kRawStagesMx - 1>();  // the scale group has landed
+        // per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
+        uint32_t mx = 0;
+        for (int i = 0; i < sr; i += 4) mx = __vmaxu4(mx, *reinterpret_cast<const uint32_t*>(my_sc + i));
+        mx = __vmaxu4(mx, mx >> 16);
+        mx = __vmaxu4(mx, mx >> 8);
+        const int crow = max(0, (int)(mx & 0xFFu) - 140);
+        s_crow[un_a & 3][t][r] = (int16_t)crow;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          uint4 n0 = c0, n1 = c1;
-          uint32_t nsc = sc;
-          if (kb + 1 < nkb) {  // next k-block's codes and scales in flight during this one
-            n0 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32));
-            n1 = __ldg(reinterpret_cast<const uint4*>(nib + (kb + 1) * 32) + 1);
-            nsc = *reinterpret_cast<const uint16_t*>(scl + (kb + 1) * 2);
-          }
+          if (kb + kRawStagesMx - 1 < nkb) issue(kb + kRawStagesMx - 1);
+          cp_async_commit();
+          cp_async_wait<kRawStagesMx - 1>();
+          const uint4 c0 = *reinterpret_cast<const uint4*>(nib_at(kb % kRawStagesMx, 0));
+          const uint4 c1 = *reinterpret_cast<const uint4*>(nib_at(kb % kRawStagesMx, 1));
+          const uint32_t sc = *reinterpret_cast<const uint16_t*>(my_sc + kb * 2);
           const uint32_t e0 = sc & 0xFFu, e1 = sc >> 8;
           uint32_t v[32];
           const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          if (MODE == 0) {
-            uint32_t f0 = e8m0_pre_factor(min(e0, 142u)), f1 = e8m0_pre_factor(min(e1, 142u));
-            // exponents above 142 do not fit one bf16 factor: apply 2^127 then the rest
-            const bool any_big = __any_sync(0xffffffffu, e0 > 142u || e1 > 142u);
-            const uint32_t g0 = e8m0_pre_factor(e0 > 142u ? e0 - 127u : 15u);
-            const uint32_t g1 = e8m0_pre_factor(e1 > 142u ? e1 - 127u : 15u);
+          const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
+          const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 8; ++c) {
+            uint32_t hv[4];
+            e2m1x8_to_f16x2(wds[c], hv);
 #pragma unroll
-              for (int b = 0; b < 4; ++b)
-                v[4 * c + b] = hmul2_bf16(e2m1x2_to_bf16x2_pre((wds[c] >> (8 * b)) & 0xFFu), c < 4 ? f0 : f1);
-            }
-            if (any_big) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = hmul2_bf16(v[i], i < 16 ? g0 : g1);
-            }
-          } else {
-            const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
-            const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t hv[4];
-              e2m1x8_to_f16x2(wds[c], hv);
-#pragma unroll
-              for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
-            }
+            for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
           }
           const int s = it % kTcStages;
           if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
@@ -345,24 +351,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
-          c0 = n0; c1 = n1; sc = nsc;
         }
       } else {
         // bf16 rows, copied as they are; column = k mod a_cols
-        const uint4* row = reinterpret_cast<const uint4*>(blob + (int64_t)R * args.a_cols * 2);
-        uint4 cur[8], nxt[8];
+        const uint8_t* row = blob + (int64_t)R * args.a_cols * 2;
+        auto chunk_at = [&](int st, int c) { return s_raw + ((st * 8 + c) * kTcAThreads + tslot) * 16; };
+        auto issue = [&](int kb2) {
+          const uint8_t* src = row + (int64_t)((kb2 * kTcKB) % args.a_cols) * 2;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cur[i] = __ldg(row + i);
+          for (int c = 0; c < 8; ++c) cp_async16(chunk_at(kb2 % kRawStagesBf, c), src + c * 16);
+        };
+#pragma unroll
+        for (int p = 0; p < kRawStagesBf - 1; ++p) {
+          if (p < nkb) issue(p);
+          cp_async_commit();
+        }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          if (kb + 1 < nkb) {
-            const int c16 = (((kb + 1) * kTcKB) % args.a_cols) / 8;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) nxt[i] = __ldg(row + c16 + i);
-          }
+          if (kb + kRawStagesBf - 1 < nkb) issue(kb + kRawStagesBf - 1);
+          cp_async_commit();
+          cp_async_wait<kRawStagesBf - 1>();
           uint32_t v[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[4 * i] = cur[i].x; v[4 * i + 1] = cur[i].y; v[4 * i + 2] = cur[i].z; v[4 * i + 3] = cur[i].w;
+          for (int c = 0; c < 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(chunk_at(kb % kRawStagesBf, c));
+            v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
           }
           const int s = it % kTcStages;
           if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
@@ -372,10 +384,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
         }
       }
+      cp_async_wait<0>();
     }
   } else if (warp == 12) {
     // ------------------------------ token producer ---------------------------
@@ -414,9 +425,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
       const int n16 = (n + 15) & ~15;
-      // bf16 operands except the routed down projection, which runs in f16
-      const uint32_t idesc =
-          (AF == kAMxfp4 && MODE == 1) ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
+      // MXFP4 weights run as f16 x f16, bf16 weights as bf16 x bf16
+      const uint32_t idesc = AF == kAMxfp4 ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
       if (lane == 0) {
         if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) give_up();
         tc_fence_after();
@@ -459,16 +469,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&acc_full, un & 1)) { give_up(); break; }
       tc_fence_after();
       const uint32_t lrow = (uint32_t)(q * 32) << 16;
-      // MXFP4 down: undo the A producer's per-row offset 2^c_r
+      // MXFP4: undo the A producer's per-row offsets 2^c_r (rows of acc0 and acc1).
+      // The producer of a unit's rows wrote them before its first k-block,
+      // which precedes acc_full; it cannot be four units ahead of this read.
       float s0 = 1.f, s1 = 1.f;
-      if (MODE == 1 && AF == kAMxfp4) {
-        const uint8_t* blob = args.w0 + (int64_t)e * args.expert_bytes + (int64_t)args.rows * (args.a_cols / 2);
-        const int cr0 =
-            max(0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + r) * (args.a_cols / 32), args.a_cols / 32) - 140);
-        const int cr1 = max(
-            0, (int)row_max_e8m0(blob + (int64_t)(mt * 256 + 128 + r) * (args.a_cols / 32), args.a_cols / 32) - 140);
-        s0 = __uint_as_float((uint32_t)(cr0 + 127) << 23);
-        s1 = __uint_as_float((uint32_t)(cr1 + 127) << 23);
+      if (AF == kAMxfp4) {
+        s0 = __uint_as_float((uint32_t)(s_crow[un & 3][0][r] + 127) << 23);
+        s1 = __uint_as_float((uint32_t)(s_crow[un & 3][1][r] + 127) << 23);
       }
       for (int c0 = 0; c0 < n; c0 += 16) {
         uint32_t g[16], h[16];
@@ -480,7 +487,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (c0 + j < n) {
-              const float hv = silu_clamped_swiglu(__uint_as_float(g[j]), __uint_as_float(h[j]), args.limit);
+              const float hv =
+                  silu_clamped_swiglu(__uint_as_float(g[j]) * s0, __uint_as_float(h[j]) * s1, args.limit);
               const int64_t o = (int64_t)(pos0 + c0 + j);
               if (AF == kAMxfp4) {
                 static_cast<__half*>(args.out)[o * args.rows + col] = __float2half_rn(hv);
@@ -513,6 +521,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tbase, kTcTmemCols);
+  }
+}
+
+// Activations bf16 -> f16 (n8 groups of 8, 16-byte aligned): exact for
+// |x| in [2^-14, 65504], f16 subnormals below; |x| > 65504 is out of range.
+__global__ void bf16_to_f16_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = in[i];
+    out[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
   }
 }
 

@@ -50,32 +50,88 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Row-major bf16 [rows][cols] viewed by TMA with a {64, 1} box and 128-byte swizzle
-// (the gather4 operand layout of the tensor-core expert kernel).
+// Row-major 16-bit [rows][cols] viewed by TMA with a {64, 16} box and 128-byte
+// swizzle (the token-operand layout of the tensor-core expert kernel).
 bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
                   CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTcBoxRows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view of a weight array for the expert kernel's loader: {row bytes of
+// the E2M1 plane, rows, experts} for MXFP4 (box {min(128, cols/2), 128, 1},
+// swizzle matching the box's inner extent), {columns, rows, 1} for a bf16
+// matrix (box {64, 128, 1}, 128-byte swizzle).
+bool make_weight_map(CUtensorMap* map, const uint8_t* base, int af, const TcArgs& a) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr || base == nullptr) return false;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  CUtensorMapDataType type;
+  CUtensorMapSwizzle swizzle;
+  if (af == kAMxfp4) {
+    dims[0] = (cuuint64_t)a.a_cols / 2;
+    dims[1] = (cuuint64_t)a.rows;
+    dims[2] = (cuuint64_t)(a.offsets != nullptr ? a.E : 1);
+    strides[0] = (cuuint64_t)a.a_cols / 2;
+    strides[1] = (cuuint64_t)a.expert_bytes;
+    box[0] = (cuuint32_t)a.w_inner;
+    type = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    swizzle = a.w_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+              : a.w_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : CU_TENSOR_MAP_SWIZZLE_32B;
+  } else {
+    dims[0] = (cuuint64_t)a.a_cols;
+    dims[1] = (cuuint64_t)a.rows;
+    dims[2] = 1;
+    strides[0] = (cuuint64_t)a.a_cols * 2;
+    strides[1] = (cuuint64_t)a.a_cols * 2 * a.rows;
+    box[0] = 64;
+    type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  }
+  box[1] = 128;
+  box[2] = 1;
+  return fn(map, type, 3, const_cast<uint8_t*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Plans the pipeline of one tensor-core expert launch, builds its weight
+// tensor maps and launches it (one CTA per SM).
 template <int MODE, int AF>
-moe_status launch_tc(const CUtensorMap& map, const TcArgs& a, cudaStream_t s) {
+moe_status launch_tc(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kTcSmemMax) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured = true;
   }
-  tc_expert_kernel<MODE, AF><<<sm_count(), kTcThreads, kTcSmem, s>>>(map, a);
+  if (!tc_plan(a, AF)) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap w0, w1;
+  if (!make_weight_map(&w0, a.w0, AF, a)) return MOE_ERR_CUDA;
+  if (MODE == 0) {
+    if (!make_weight_map(&w1, a.w1, AF, a)) return MOE_ERR_CUDA;
+  } else {
+    w1 = w0;
+  }
+  tc_expert_kernel<MODE, AF><<<sm_count(), kTcThreads, a.smem_bytes, s>>>(bmap, w0, w1, a);
   return launch_status();
+}
+
+// Tokens per expert-kernel unit: the accumulator columns a unit reserves.  A
+// small chunk (few pairs per expert) leaves TMEM and shared memory for deeper
+// rings; a chunk below an expert's pair count makes its weights stream again.
+int expert_chunk(int T, int K, int E) {
+  const int64_t avg = ((int64_t)T * K + E - 1) / E;
+  return avg <= 8 ? 32 : avg <= 24 ? 64 : kTcNMax;
 }
 
 // Router and shared expert run on the tensor cores above this token count
@@ -269,8 +325,9 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  // x in f16 [T][hidden], then h in f16 [T*top_k][inter]
-  return round_up((size_t)T * dims->hidden * 2, 256) + round_up((size_t)T * dims->top_k * dims->inter * 2, 256);
+  // x in pair order and f16 [T*top_k][hidden], then h in f16 [T*top_k][inter]
+  const size_t pairs = (size_t)T * dims->top_k;
+  return round_up(pairs * dims->hidden * 2, 256) + round_up(pairs * dims->inter * 2, 256);
 }
 
 moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
@@ -290,16 +347,9 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
+  const int64_t pairs = (int64_t)T * dims->top_k;
   __half* x16 = static_cast<__half*>(ws);
-  __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)T * H * 2, 256));
-  const int64_t n8 = (int64_t)T * H / 8;
-  bf16_to_f16_kernel<<<(int)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184), 256, 0, s>>>(
-      static_cast<const uint4*>(x), reinterpret_cast<uint4*>(x16), n8);
-  if ((st = launch_status()) != MOE_OK) return st;
-  CUtensorMap xmap, hmap;
-  if (!make_row_map(&xmap, x16, T, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_row_map(&hmap, h16, (int64_t)T * dims->top_k, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
-    return MOE_ERR_CUDA;
+  __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)pairs * H * 2, 256));
   TcArgs g{};
   g.w0 = gate.base;
   g.w1 = up.base;
@@ -309,13 +359,10 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   g.k_total = H;
   g.b_cols = H;
   g.offsets = offsets;
-  g.perm = perm;
-  g.K = dims->top_k;
   g.E = dims->n_experts;
-  g.n_chunk = kTcNMax;
+  g.n_chunk = expert_chunk(T, dims->top_k, dims->n_experts);
   g.out = h16;
   g.limit = dims->swiglu_limit;
-  if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
   TcArgs d = g;
   d.w0 = down.base;
   d.w1 = nullptr;
@@ -324,8 +371,22 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   d.a_cols = I;
   d.k_total = I;
   d.b_cols = I;
-  d.perm = nullptr;
   d.out = y_perm;
+  {  // shape check before anything is enqueued
+    TcArgs pg = g, pd = d;
+    if (!tc_plan(pg, kAMxfp4) || !tc_plan(pd, kAMxfp4)) return MOE_ERR_UNSUPPORTED;
+  }
+  // the activations of every pair, in expert order and f16 (the token operand
+  // of the gate/up GEMM is then read with plain TMA boxes)
+  const int64_t n8 = pairs * H / 8;
+  gather_f16_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
+      static_cast<const uint4*>(x), perm, dims->top_k, H / 8, pairs, reinterpret_cast<uint4*>(x16));
+  if ((st = launch_status()) != MOE_OK) return st;
+  CUtensorMap xmap, hmap;
+  if (!make_row_map(&xmap, x16, pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_row_map(&hmap, h16, pairs, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MOE_ERR_CUDA;
+  if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
   return launch_tc<1, kAMxfp4>(hmap, d, s);
 }
 

@@ -1,7 +1,7 @@
-// Grouped expert GEMM on the 5th-generation tensor cores (tcgen05), for the
-// prefill / many-token regime.
+// Grouped expert GEMM on the 5th-generation tensor cores (tcgen05), for every
+// token count.
 //
-// Per unit = (expert e, token chunk of <= 128 grouped pairs, 128-row tile):
+// Per unit = (expert e, token chunk of <= n_chunk grouped pairs, row tile):
 //   MODE 0 (gate/up):  acc0 = Wg[rows] x^T, acc1 = Wu[rows] x^T over K = hidden;
 //                      epilogue h = silu(min(acc0, L)) * clamp(acc1, -L, L),
 //                      stored in f16 (|h| <= L^2; 11 mantissa bits)
@@ -11,30 +11,41 @@
 // c_r), c_r = max(0, e_max(row) - 140), with 2^c_r applied to the fp32
 // accumulator row in the epilogue.  That is exact whenever a row's E8M0
 // exponents span at most 36 octaves, and costs two instructions per pair of
-// codes (cvt + multiply), which keeps the tensor cores, not the dequant, the
-// limit.  bf16 weights (shared expert, router) are copied as they are.
+// codes (cvt + multiply).  bf16 weights (shared expert, router) are copied as
+// they are.
 // ("Model techniques map", row "SwiGLU feed-forward": the clamped SwiGLU;
 // "ElytronAI / DeepSeek-v4-Flash", Sizes/Layout: MXFP4 weights, expert xid at
 // base + xid * expert_bytes.)
 //
 // Swap-AB: the weight rows are the MMA's M = 128 dimension and the expert's
-// tokens its N dimension (a multiple of 16, <= 128), so a unit needs no token
-// padding beyond 16.
+// tokens its N dimension (a multiple of 16, <= n_chunk), so a unit needs no
+// token padding beyond 16.  The token operand is read from a matrix already in
+// unit order (activations gathered per pair beforehand, or h), so it arrives
+// by plain 2-D TMA boxes.
 //
-// Roles (448 threads, one CTA per SM, persistent over units):
+// Pipeline stage = 2 k-blocks of 64 (K = 128): the A producers write both
+// k-blocks' values to TMEM, the token loader both k-blocks' token tiles, and
+// the MMA issuer runs 16 MMAs and ONE tcgen05.commit per stage.  On B200 every
+// producer/consumer handshake around the tensor pipe costs a few hundred
+// cycles that do not overlap the MMAs, so stages are made as long as TMEM
+// allows.
+//
+// Roles (480 threads, one CTA per SM, persistent over units):
 //   warps 0-3   epilogue: tcgen05.ld of the two accumulators (TMEM lane
 //               quadrant = warp), SwiGLU or copy, global stores;
-//   warps 4-11  A producer: thread = one weight row of one of the two tiles;
-//               its raw k-blocks arrive through a private cp.async ring; per
-//               64-column k-block it converts the 32 code bytes exactly (see
-//               above) and writes the 64 values into TMEM with tcgen05.st: the
-//               MMA takes its A operand from TMEM, so the weight tiles never
-//               touch shared memory;
-//   warp 12     token producer: TMA tile::gather4 of the unit's activation rows
-//               (bf16, 128-byte swizzle) into a 4-stage shared-memory ring;
-//   warp 13     TMEM owner and MMA issuer (one thread): 2 x 4 tcgen05.mma
-//               (M=128, N=n16, K=16) per k-block, tcgen05.commit to free stages.
-// TMEM (512 columns): acc0 [0,128), acc1 [128,256), A stages [256, 512).
+//   warps 4-11  A producers: thread = one weight row of one of the two tiles;
+//               reads its row's bytes from the weight ring (conflict-free: the
+//               ring holds swizzled TMA boxes), converts them exactly and writes
+//               them into TMEM with tcgen05.st: the MMA takes A from TMEM.
+//               Each thread fetches its row's E8M0 bytes for the NEXT unit with
+//               cp.async into a thread-major buffer;
+//   warp 12     token loader: 2-D TMA boxes of 16 token rows x 64 columns;
+//   warp 13     TMEM owner and MMA issuer (one thread);
+//   warp 14     weight loader (one thread): 3-D TMA boxes (128 rows x <= 128
+//               bytes per tile, expert index as the third coordinate) into the
+//               weight ring, running ahead across unit boundaries.
+// TMEM (512 columns): acc0 [0, acc), acc1 [acc, 2 acc), stages of 128 columns
+// (2 k-blocks x 2 tiles x 32) from 2 acc.
 #pragma once
 
 #include <cuda.h>
@@ -43,35 +54,30 @@
 
 namespace moe {
 
-constexpr int kTcThreads = 448;
-constexpr int kTcStages = 4;
-constexpr int kTcKB = 64;     // k per stage (one 128-byte swizzle atom of bf16)
-constexpr int kTcNMax = 128;  // tokens per unit
-constexpr int kTcBTile = kTcNMax * kTcKB * 2;  // 16 KB per stage
+constexpr int kTcThreads = 480;
+constexpr int kTcKB = 64;      // k per k-block (one 128-byte swizzle atom of 16-bit values)
+constexpr int kTcKG = 2;       // k-blocks per pipeline stage
+constexpr int kTcStageK = kTcKB * kTcKG;
+constexpr int kTcNMax = 128;   // tokens per unit
 constexpr int kTcTmemCols = 512;
-constexpr int kTcAccCols = 128;
-constexpr int kTcAStage = 64;  // TMEM columns per stage: 2 tiles x 32
-// Raw A staging: every A-producer thread copies its own weight row's next
-// k-blocks with cp.async into a private ring, kRawStagesMx deep for MXFP4
-// (32 code bytes per k-block; the row's whole E8M0 row is fetched once per
-// unit) and kRawStagesBf deep for bf16 rows (128 bytes per k-block).  Code
-// planes are [stage][16-byte chunk][thread], so a warp's 16-byte reads are
-// contiguous.
-constexpr int kTcAThreads = 256;
-constexpr int kRawStagesMx = 6;
-constexpr int kRawStagesBf = 3;
-constexpr int kScaleRowMax = 128;  // E8M0 bytes per weight row held per producer thread (cols <= 4096)
-constexpr int kRawMxBytes = kRawStagesMx * 2 * kTcAThreads * 16 + kTcAThreads * kScaleRowMax;  // 80 KB
-constexpr int kRawBfBytes = kRawStagesBf * 8 * kTcAThreads * 16;                          // 96 KB
-constexpr int kRawBytes = kRawMxBytes > kRawBfBytes ? kRawMxBytes : kRawBfBytes;
-constexpr int kTcSmemUsed = kTcStages * kTcBTile + kRawBytes + 1024 /*align*/ + 8192 /*tables*/;
-// requested dynamic shared memory: more than half an SM's, so one CTA per SM
-// (each CTA owns all 512 TMEM columns)
-constexpr int kTcSmem = kTcSmemUsed;
-static_assert(kTcSmem > 114 * 1024 && kTcSmem <= 227 * 1024, "tc_expert shared memory");
+constexpr int kTcStageCols = 64 * kTcKG;  // TMEM columns of one stage
+constexpr int kTcMaxStages = 8;  // upper bound of every ring's depth
+constexpr int kTcAThreads = 256; // A producer threads (8 warps)
+constexpr int kTcBoxRows = 16;   // token rows per TMA box
+constexpr int kCrowRing = 8;     // units of per-row offsets kept for the epilogue
+constexpr int kScaleRowMax = 128;  // E8M0 bytes per weight row (cols <= 4096)
+// Dynamic shared memory one CTA may use (the opt-in maximum minus the static
+// arrays and the alignment slack).
+constexpr int kTcSmemMax = 227 * 1024 - 6 * 1024;
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -136,17 +142,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Four rows (r0..r3), 64 bf16 columns from col, of a 2-D tensor map whose box
-// is {64, 1} with 128-byte swizzle, into 512 contiguous bytes of shared memory.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int col, int r0, int r1, int r2,
-                                            int r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, "
-      "{%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 B apart (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
@@ -166,17 +161,48 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Box {x, y, z} of a 3-D tensor map into shared memory, L2 hint `policy`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Box {x, y} of a 2-D tensor map into shared memory.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // f16x2 with 2^k in both halves, k in [-24, 15] (subnormal f16 below -14).
 __device__ __forceinline__ uint32_t pow2_f16x2(int k) {
   const float f = __uint_as_float((uint32_t)(k + 127) << 23);
   return f32x2_to_f16x2(f, f);
 }
 
-__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
+// Byte offset inside a TMA box written with the swizzle mode that matches its
+// inner extent (128 B: SWIZZLE_128B, 64 B: SWIZZLE_64B): the 16-byte chunk
+// bits [4, 4+b) are XORed with the row bits [7, 7+b), mask = 2^b - 1.
+__device__ __forceinline__ uint32_t swz(uint32_t off, uint32_t mask) { return off ^ (((off >> 7) & mask) << 4); }
+
+// Slot and phase of a ring of `n` stages.
+struct TcRing {
+  int s, n;
+  uint32_t ph;
+  __device__ explicit TcRing(int depth) : s(0), n(depth), ph(0) {}
+  __device__ void next() {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1;
+    }
+  }
+};
 
 enum { kAMxfp4 = 0, kABf16 = 1 };
 
@@ -187,36 +213,94 @@ struct TcArgs {
   int rows;              // rows of one projection (the MMA's M extent)
   int a_cols;            // columns of the weight matrix
   int k_total;           // reduction length: a multiple of a_cols (A column = k mod a_cols)
-  int b_cols;            // columns of a B row (B column = k mod b_cols)
-  const int32_t* offsets;  // [E+1] grouped pairs; null: one group of n_single rows
-  const int32_t* perm;     // B row of pos = perm[pos] / K; null: B row = pos
-  int K, E, n_single;
+  int b_cols;            // columns of a token row (token column = k mod b_cols)
+  const int32_t* offsets;  // [E+1] grouped rows; null: one group of n_single rows
+  int E, n_single;
   int n_chunk;           // tokens per unit: multiple of 16, <= kTcNMax
   void* out;             // see the epilogue
   float limit;
+  // pipeline shape, filled in by tc_plan()
+  int acc_cols;      // TMEM columns per accumulator (>= n_chunk)
+  int stages;        // pipeline stages (TMEM A + token tiles of 2 k-blocks)
+  int w_slots;       // weight slots
+  int w_inner;       // bytes of one weight row in one TMA box
+  int w_slot_bytes;  // bytes of one weight slot (both tiles)
+  int st_per_slot;   // pipeline stages per weight slot
+  int sr;            // E8M0 bytes per weight row (MXFP4)
+  int off_b, off_sc, off_prefix;  // shared-memory offsets from the 1024-aligned base
+  int smem_bytes;                 // dynamic shared memory of the launch
 };
+
+// Ring depths and the shared-memory carve-up of one launch.  False when the
+// shape is outside what the kernel implements.
+inline bool tc_plan(TcArgs& a, int af) {
+  const int nc = a.n_chunk;
+  if (nc < 16 || nc > kTcNMax || nc % 16) return false;
+  if (a.k_total % kTcStageK || a.a_cols % kTcKB || a.b_cols % kTcKB || a.k_total % a.a_cols) return false;
+  a.acc_cols = nc <= 32 ? 32 : nc <= 64 ? 64 : 128;
+  a.stages = (kTcTmemCols - 2 * a.acc_cols) / kTcStageCols;
+  if (a.stages > kTcMaxStages) a.stages = kTcMaxStages;
+  const int nst = a.k_total / kTcStageK;
+  if (af == kAMxfp4) {
+    if (a.a_cols % kTcStageK || a.a_cols / 32 > kScaleRowMax || a.k_total != a.a_cols) return false;
+    a.w_inner = a.a_cols / 2 < 128 ? a.a_cols / 2 : 128;
+    if ((a.a_cols / 2) % a.w_inner) return false;
+    a.st_per_slot = a.w_inner / 64;  // 64 code bytes of a row per stage
+    a.w_slot_bytes = 2 * 128 * a.w_inner;
+    a.sr = a.a_cols / 32;
+  } else {
+    a.w_inner = 128;  // 64 bf16 columns per box, two boxes per tile and stage
+    a.st_per_slot = 1;
+    a.w_slot_bytes = 2 * kTcKG * 128 * 128;
+    a.sr = 0;
+  }
+  if (nst % a.st_per_slot) return false;
+  // the A producers run at most ceil(stages / nst) + 1 units ahead of the
+  // epilogue, which reads their per-row offsets
+  if ((a.stages + nst - 1) / nst + 1 >= kCrowRing) return false;
+  const int bst = kTcKG * nc * 128;
+  const int sc = af == kAMxfp4 ? 2 * kTcAThreads * a.sr : 0;
+  const int groups = a.offsets != nullptr ? a.E : 1;
+  const int pre = ((groups + 1) * 4 + 127) / 128 * 128;
+  const int budget = kTcSmemMax - 1024;  // 1024: alignment slack of the dynamic base
+  const int w = (budget - a.stages * bst - sc - pre) / a.w_slot_bytes;
+  a.w_slots = w < 6 ? w : 6;
+  if (a.w_slots < 2) return false;
+  a.off_b = a.w_slots * a.w_slot_bytes;
+  a.off_sc = a.off_b + a.stages * bst;
+  a.off_prefix = a.off_sc + sc;
+  a.smem_bytes = a.off_prefix + pre + 1024;
+  return a.smem_bytes <= kTcSmemMax;
+}
 
 template <int MODE, int AF>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs args) {
+    tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap0,
+                     const __grid_constant__ CUtensorMap wmap1, const TcArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t a_full[kTcStages], b_full[kTcStages], empty[kTcStages];
-  __shared__ __align__(8) uint64_t acc_full, acc_empty;
+  __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages], b_full[kTcMaxStages];
+  __shared__ __align__(8) uint64_t w_full[kTcMaxStages], w_empty[kTcMaxStages];
+  __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
   __shared__ uint32_t s_taddr;
   __shared__ int32_t s_abort;
-  __shared__ int32_t s_rows[kTcNMax];
-  __shared__ int16_t s_crow[4][2][128];  // per-row f16 offsets c_r, ring over units
+  __shared__ int16_t s_crow[kCrowRing][2][128];  // per-row f16 offsets c_r, ring over units
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_raw = smem + kTcStages * kTcBTile;                                    // raw A ring
-  int32_t* s_prefix = reinterpret_cast<int32_t*>(s_raw + kRawBytes);               // [E + 1]
+  uint8_t* s_w = smem;                  // weight ring
+  uint8_t* s_b = smem + args.off_b;     // token tiles, one per stage
+  uint8_t* s_sc = smem + args.off_sc;   // E8M0 rows, two unit buffers, thread-major
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + args.off_prefix);  // [E + 1]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool grouped = args.offsets != nullptr;
   const int E = grouped ? args.E : 1;
   const int MT = MODE == 0 ? args.rows / 128 : args.rows / 256;  // row tiles per group
-  const int nkb = args.k_total / kTcKB;
+  const int nst = args.k_total / kTcStageK;                       // stages per unit
   const int NC = args.n_chunk;
+  const int tile_bytes = args.w_slot_bytes / 2;
+  const int atom = NC * 128;         // one k-block of token rows (128-byte rows)
+  const int bst = kTcKG * atom;      // token bytes of one stage
+  const uint32_t a_base = 2 * args.acc_cols;
 
   // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
   if (warp == 0) {
@@ -240,13 +324,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) s_prefix[E] = run;
   }
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&a_full[s], 8);
-      mbar_init(&b_full[s], 1);
+    for (int s = 0; s < kTcMaxStages; ++s) {
+      mbar_init(&full[s], 8);  // one arrival per A-producer warp (one of them also waits for the tokens)
       mbar_init(&empty[s], 1);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&w_full[s], 1);
+      mbar_init(&w_empty[s], 8);
     }
     mbar_init(&acc_full, 1);
     mbar_init(&acc_empty, 4);
+    mbar_init(&mma_done, 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -260,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tbase = s_taddr;
   const int n_units = s_prefix[E];
 
-  // unit -> (group, row tile, first position, tokens)
+  // unit -> (group, row tile, first row of the token matrix, tokens)
   auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {  // last e with s_prefix[e] <= u
@@ -283,59 +370,83 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp >= 4 && warp < 12) {
-    // ------------------------------ A producer ---------------------------------
+    // ------------------------------ A producers --------------------------------
     const int t = (warp - 4) >> 2, q = warp & 3, r = q * 32 + lane;
-    uint32_t it = 0, un_a = 0;
-    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un_a) {
-      int e, mt, pos0, n;
-      decode_unit(u, e, mt, pos0, n);
-      const int R = MODE == 0 ? mt * 128 + r : mt * 256 + t * 128 + r;
-      const uint8_t* blob = (MODE == 0 && t == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes;
-      const int tslot = (warp - 4) * 32 + lane;
-      if (AF == kAMxfp4) {
-        const uint8_t* nib = blob + (int64_t)R * (args.a_cols / 2);
-        const int sr = args.a_cols / 32;  // scale bytes per row (multiple of 4, <= kScaleRowMax)
-        const uint8_t* scl = blob + (int64_t)args.rows * (args.a_cols / 2) + (int64_t)R * sr;
-        uint8_t* my_sc = s_raw + kRawStagesMx * 2 * kTcAThreads * 16 + tslot * kScaleRowMax;
-        auto nib_at = [&](int st, int h) { return s_raw + ((st * 2 + h) * kTcAThreads + tslot) * 16; };
-        auto issue = [&](int kb2) {
-          cp_async16(nib_at(kb2 % kRawStagesMx, 0), nib + kb2 * 32);
-          cp_async16(nib_at(kb2 % kRawStagesMx, 1), nib + kb2 * 32 + 16);
-        };
-        // the row's E8M0 bytes in one go (first group), then the ring prologue
-        if (sr % 16 == 0) {
-          for (int i = 0; i < sr; i += 16) cp_async16(my_sc + i, scl + i);
-        } else {
-          for (int i = 0; i < sr; i += 4)
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(my_sc + i)), "l"(scl + i)
-                         : "memory");
+    const int tslot = (warp - 4) * 32 + lane;
+    const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + a_base + t * 32;
+    const uint32_t mask = (uint32_t)args.w_inner / 16 - 1;
+    TcRing rs(args.stages), rw(args.w_slots);
+    int js = 0;  // stage within the current weight slot
+    // publish stage rs.s (both k-blocks stored): the tokens of the stage must
+    // have landed too (warp 4 checks), then one arrival per warp
+    auto publish = [&]() -> bool {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      bool ok = true;
+      if (warp == 4 && lane == 0) ok = mbar_wait(&b_full[rs.s], rs.ph);
+      if (lane == 0) mbar_arrive(&full[rs.s]);
+      rs.next();
+      if (++js == args.st_per_slot) {  // slot fully read: hand it back to the loader
+        js = 0;
+        if (lane == 0) mbar_arrive(&w_empty[rw.s]);
+        rw.next();
+      }
+      return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    };
+    auto wait_stage = [&]() -> bool {  // TMEM stage free (its MMAs done)
+      if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) return false;
+      tc_fence_after();
+      return true;
+    };
+    if (AF == kAMxfp4) {
+      const int sr = args.sr, cs = sr < 16 ? sr : 16;
+      const int64_t plane = (int64_t)args.rows * (args.a_cols / 2);
+      // this thread's E8M0 row of unit u -> scale buffer `buf`, cs-byte pieces
+      // at [piece][thread] (cp.async; committed by the caller)
+      auto sc_issue = [&](int u, int buf) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        const int R = MODE == 0 ? mt * 128 + r : mt * 256 + t * 128 + r;
+        const uint8_t* src =
+            (MODE == 0 && t == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes + plane + (int64_t)R * sr;
+        uint8_t* dst = s_sc + buf * kTcAThreads * sr + tslot * cs;
+        for (int c = 0; c < sr / cs; ++c) {
+          uint8_t* d = dst + c * kTcAThreads * cs;
+          if (cs == 16) cp_async16(d, src + c * 16);
+          else if (cs == 8) cp_async8(d, src + c * 8);
+          else cp_async4(d, src + c * 4);
         }
+      };
+      if ((int)blockIdx.x < n_units) sc_issue(blockIdx.x, 0);
+      cp_async_commit();
+      uint32_t un = 0;
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+        if (u + (int)gridDim.x < n_units) sc_issue(u + gridDim.x, (un + 1) & 1);
         cp_async_commit();
-#pragma unroll
-        for (int p = 0; p < kRawStagesMx - 1; ++p) {
-          if (p < nkb) issue(p);
-          cp_async_commit();
-        }
-        cp_async_wait<kRawStagesMx - 1>();  // the scale group has landed
+        cp_async_wait<1>();  // this unit's E8M0 row has landed
+        const uint8_t* scb = s_sc + (un & 1) * kTcAThreads * sr + tslot * cs;
+        auto sc_word = [&](int w) {  // E8M0 bytes 4w .. 4w + 3 of the row
+          const int b = 4 * w;
+          return *reinterpret_cast<const uint32_t*>(scb + (b / cs) * kTcAThreads * cs + b % cs);
+        };
         // per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
         uint32_t mx = 0;
-        for (int i = 0; i < sr; i += 4) mx = __vmaxu4(mx, *reinterpret_cast<const uint32_t*>(my_sc + i));
+        for (int w = 0; w < sr / 4; ++w) mx = __vmaxu4(mx, sc_word(w));
         mx = __vmaxu4(mx, mx >> 16);
         mx = __vmaxu4(mx, mx >> 8);
         const int crow = max(0, (int)(mx & 0xFFu) - 140);
-        s_crow[un_a & 3][t][r] = (int16_t)crow;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          if (kb + kRawStagesMx - 1 < nkb) issue(kb + kRawStagesMx - 1);
-          cp_async_commit();
-          cp_async_wait<kRawStagesMx - 1>();
-          const uint4 c0 = *reinterpret_cast<const uint4*>(nib_at(kb % kRawStagesMx, 0));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(nib_at(kb % kRawStagesMx, 1));
-          const uint32_t sc = *reinterpret_cast<const uint16_t*>(my_sc + kb * 2);
-          const uint32_t e0 = sc & 0xFFu, e1 = sc >> 8;
-          uint32_t v[32];
+        s_crow[un % kCrowRing][t][r] = (int16_t)crow;
+        // k-block g of the current stage of this row -> 64 f16 values
+        auto convert = [&](int g, uint32_t sw, uint32_t (&v)[32]) {
+          const uint8_t* tile = s_w + rw.s * args.w_slot_bytes + t * tile_bytes;
+          const uint32_t o = (uint32_t)(r * args.w_inner + 64 * js + 32 * g);
+          const uint4 c0 = *reinterpret_cast<const uint4*>(tile + swz(o, mask));
+          const uint4 c1 = *reinterpret_cast<const uint4*>(tile + swz(o + 16, mask));
+          const int e0 = (int)((sw >> (16 * g)) & 0xFFu), e1 = (int)((sw >> (16 * g + 8)) & 0xFFu);
           const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          const uint32_t f0 = pow2_f16x2(max((int)e0 - 127 - crow, -24));
-          const uint32_t f1 = pow2_f16x2(max((int)e1 - 127 - crow, -24));
+          const uint32_t f0 = pow2_f16x2(max(e0 - 127 - crow, -24));
+          const uint32_t f1 = pow2_f16x2(max(e1 - 127 - crow, -24));
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t hv[4];
@@ -343,119 +454,196 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int b = 0; b < 4; ++b) v[4 * c + b] = hmul2(hv[b], c < 4 ? f0 : f1);
           }
-          const int s = it % kTcStages;
-          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
-          tc_fence_after();
-          tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[s]);
-        }
-      } else {
-        // bf16 rows, copied as they are; column = k mod a_cols
-        const uint8_t* row = blob + (int64_t)R * args.a_cols * 2;
-        auto chunk_at = [&](int st, int c) { return s_raw + ((st * 8 + c) * kTcAThreads + tslot) * 16; };
-        auto issue = [&](int kb2) {
-          const uint8_t* src = row + (int64_t)((kb2 * kTcKB) % args.a_cols) * 2;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) cp_async16(chunk_at(kb2 % kRawStagesBf, c), src + c * 16);
         };
-#pragma unroll
-        for (int p = 0; p < kRawStagesBf - 1; ++p) {
-          if (p < nkb) issue(p);
-          cp_async_commit();
-        }
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          if (kb + kRawStagesBf - 1 < nkb) issue(kb + kRawStagesBf - 1);
-          cp_async_commit();
-          cp_async_wait<kRawStagesBf - 1>();
-          uint32_t v[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(chunk_at(kb % kRawStagesBf, c));
-            v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
+        bool ok = true;
+        for (int st = 0; st < nst && ok; ++st) {
+          if (js == 0 && !mbar_wait(&w_full[rw.s], rw.ph)) {
+            ok = false;
+            break;
           }
-          const int s = it % kTcStages;
-          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); break; }
-          tc_fence_after();
-          tmem_st32(tbase + ((uint32_t)(q * 32) << 16) + kTcTmemCols / 2 + s * kTcAStage + t * 32, v);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[s]);
+          const uint32_t sw = sc_word(st);  // E8M0 of this stage's two k-blocks
+          uint32_t v0[32], v1[32];
+          convert(0, sw, v0);
+          if (!wait_stage()) {
+            ok = false;
+            break;
+          }
+          tmem_st32(tl + rs.s * kTcStageCols, v0);
+          convert(1, sw, v1);
+          tmem_st32(tl + rs.s * kTcStageCols + 64, v1);
+          ok = publish();
+        }
+        if (!ok) {
+          give_up();
+          break;
         }
       }
       cp_async_wait<0>();
-    }
-  } else if (warp == 12) {
-    // ------------------------------ token producer ---------------------------
-    uint32_t it = 0;
-    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
-      int e, mt, pos0, n;
-      decode_unit(u, e, mt, pos0, n);
-      const int n16 = (n + 15) & ~15;
-      for (int j = lane; j < n16; j += 32) {
-        const int p = pos0 + min(j, n - 1);  // pad rows repeat the last token
-        s_rows[j] = args.perm != nullptr ? args.perm[p] / args.K : p;
-      }
-      __syncwarp();
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kTcStages;
-        if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1)) { give_up(); }
-          else {
-            mbar_arrive_expect_tx(&b_full[s], (uint32_t)n16 * kTcKB * 2);
-            uint8_t* dst = smem + s * kTcBTile;
-            const int col = (kb * kTcKB) % args.b_cols;
-            for (int j = 0; j < n16; j += 4)
-              tma_gather4(dst + j * 128, &bmap, col, s_rows[j], s_rows[j + 1], s_rows[j + 2], s_rows[j + 3],
-                          &b_full[s]);
-          }
+    } else {
+      // bf16 rows, copied as they are (the loader picks column k mod a_cols)
+      auto copy = [&](int g, uint32_t (&v)[32]) {
+        const uint8_t* box = s_w + rw.s * args.w_slot_bytes + t * tile_bytes + g * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(box + swz((uint32_t)(r * 128 + 16 * c), 7));
+          v[4 * c] = w.x;
+          v[4 * c + 1] = w.y;
+          v[4 * c + 2] = w.z;
+          v[4 * c + 3] = w.w;
         }
-        __syncwarp();
-        if (aborted()) break;
+      };
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        bool ok = true;
+        for (int st = 0; st < nst && ok; ++st) {
+          if (!mbar_wait(&w_full[rw.s], rw.ph)) {
+            ok = false;
+            break;
+          }
+          uint32_t v0[32], v1[32];
+          copy(0, v0);
+          if (!wait_stage()) {
+            ok = false;
+            break;
+          }
+          tmem_st32(tl + rs.s * kTcStageCols, v0);
+          copy(1, v1);
+          tmem_st32(tl + rs.s * kTcStageCols + 64, v1);
+          ok = publish();
+        }
+        if (!ok) {
+          give_up();
+          break;
+        }
       }
-      __syncwarp();
     }
+  } else if (warp == 14) {
+    // ------------------------------ weight loader ------------------------------
+    if (lane == 0) {
+      TcRing rw(args.w_slots);
+      const uint64_t pol = policy_evict_first();
+      const int n_slots = nst / args.st_per_slot;
+      int issued = 0;
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        bool ok = true;
+        const int y0 = MODE == 0 ? mt * 128 : mt * 256;
+        const int y1 = MODE == 0 ? mt * 128 : mt * 256 + 128;
+        for (int i = 0; i < n_slots; ++i) {
+          if (!mbar_wait(&w_empty[rw.s], rw.ph ^ 1)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&w_full[rw.s], (uint32_t)args.w_slot_bytes);
+          uint8_t* dst = s_w + rw.s * args.w_slot_bytes;
+          if (AF == kAMxfp4) {  // code bytes [i * w_inner, +w_inner) of 128 rows, expert e
+            tma_load_3d(dst, &wmap0, i * args.w_inner, y0, e, &w_full[rw.s], pol);
+            tma_load_3d(dst + tile_bytes, MODE == 0 ? &wmap1 : &wmap0, i * args.w_inner, y1, e, &w_full[rw.s], pol);
+          } else {  // bf16 columns (k mod a_cols) of the stage's two k-blocks
+#pragma unroll
+            for (int g = 0; g < kTcKG; ++g) {
+              const int x = (i * kTcStageK + g * kTcKB) % args.a_cols;
+              tma_load_3d(dst + g * 16384, &wmap0, x, y0, 0, &w_full[rw.s], pol);
+              tma_load_3d(dst + tile_bytes + g * 16384, MODE == 0 ? &wmap1 : &wmap0, x, y1, 0, &w_full[rw.s], pol);
+            }
+          }
+          rw.next();
+          ++issued;
+        }
+        if (!ok) break;
+      }
+      // the last fills must have landed before the CTA exits (on the normal
+      // path the A producers have already waited for every one of them)
+      for (int i = 0; i < min(issued, rw.n); ++i) {
+        const int s = (rw.s - 1 - i + rw.n) % rw.n;
+        if (!mbar_wait(&w_full[s], s < rw.s ? rw.ph : rw.ph ^ 1)) set_error(kErrWaitTc);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 12) {
+    // ------------------------------ token loader -------------------------------
+    if (lane == 0) {
+      TcRing rs(args.stages);
+      int issued = 0;
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        const int n16 = (n + 15) & ~15;  // rows past the chunk are loaded but never stored
+        bool ok = true;
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[rs.s], (uint32_t)(kTcKG * n16 * 128));
+          uint8_t* dst = s_b + rs.s * bst;
+#pragma unroll
+          for (int g = 0; g < kTcKG; ++g) {
+            const int col = (st * kTcStageK + g * kTcKB) % args.b_cols;
+            for (int j = 0; j < n16; j += kTcBoxRows)
+              tma_load_2d(dst + g * atom + j * 128, &bmap, col, pos0 + j, &b_full[rs.s]);
+          }
+          rs.next();
+          ++issued;
+        }
+        if (!ok) break;
+      }
+      for (int i = 0; i < min(issued, rs.n); ++i) {
+        const int s = (rs.s - 1 - i + rs.n) % rs.n;
+        if (!mbar_wait(&b_full[s], s < rs.s ? rs.ph : rs.ph ^ 1)) set_error(kErrWaitTc);
+      }
+    }
+    __syncwarp();
   } else if (warp == 13) {
     // ------------------------------ MMA issuer --------------------------------
-    uint32_t it = 0, un = 0;
-    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
-      int e, mt, pos0, n;
-      decode_unit(u, e, mt, pos0, n);
-      const int n16 = (n + 15) & ~15;
-      // MXFP4 weights run as f16 x f16, bf16 weights as bf16 x bf16
-      const uint32_t idesc = AF == kAMxfp4 ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
-      if (lane == 0) {
-        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) give_up();
+    if (lane == 0) {
+      TcRing rs(args.stages);
+      uint32_t un = 0;
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        const int n16 = (n + 15) & ~15;
+        // MXFP4 weights run as f16 x f16, bf16 weights as bf16 x bf16
+        const uint32_t idesc = AF == kAMxfp4 ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
+        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) {
+          give_up();
+          break;
+        }
         tc_fence_after();
-      }
-      __syncwarp();
-      for (int kb = 0; kb < nkb && !aborted(); ++kb, ++it) {
-        const int s = it % kTcStages;
-        if (lane == 0) {
-          const uint32_t ph = (it / kTcStages) & 1;
-          if (!mbar_wait(&a_full[s], ph) || !mbar_wait(&b_full[s], ph)) { give_up(); }
-          else {
-            tc_fence_after();
-            const uint32_t bsa = smem_u32(smem + s * kTcBTile);
-            const uint32_t a0 = tbase + kTcTmemCols / 2 + s * kTcAStage;
+        bool ok = true;
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(&full[rs.s], rs.ph)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t bsa = smem_u32(s_b + rs.s * bst);
+          const uint32_t a0 = tbase + a_base + rs.s * kTcStageCols;
+#pragma unroll
+          for (int g = 0; g < kTcKG; ++g) {
 #pragma unroll
             for (int ks = 0; ks < kTcKB / 16; ++ks) {
-              const uint64_t bd = sdesc_sw128(bsa + ks * 32);
-              const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-              umma_tmem_a(tbase, a0 + ks * 8, bd, idesc, acc);
-              umma_tmem_a(tbase + kTcAccCols, a0 + 32 + ks * 8, bd, idesc, acc);
+              const uint64_t bd = sdesc_sw128(bsa + g * atom + ks * 32);
+              const uint32_t acc = (st > 0 || g > 0 || ks > 0) ? 1u : 0u;
+              umma_tmem_a(tbase, a0 + g * 64 + ks * 8, bd, idesc, acc);
+              umma_tmem_a(tbase + args.acc_cols, a0 + g * 64 + 32 + ks * 8, bd, idesc, acc);
             }
-            umma_commit(&empty[s]);
-            if (kb == nkb - 1) umma_commit(&acc_full);
           }
+          umma_commit(&empty[rs.s]);
+          if (st == nst - 1) umma_commit(&acc_full);
+          rs.next();
         }
-        __syncwarp();
+        if (!ok) break;
       }
+      // every MMA of this thread done before TMEM is released
+      umma_commit(&mma_done);
+      if (!mbar_wait(&mma_done, 0)) set_error(kErrWaitTc);
     }
-  } else {
+    __syncwarp();
+  } else if (warp < 4) {
     // ------------------------------ epilogue ----------------------------------
     // MODE 0, MXFP4: h = swiglu(gate, up) in f16 [pos][rows]
     // MODE 0, bf16:  h as a bf16 pair, hi at [pos][col], lo = h - hi at [pos][rows + col]
@@ -469,18 +657,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&acc_full, un & 1)) { give_up(); break; }
       tc_fence_after();
       const uint32_t lrow = (uint32_t)(q * 32) << 16;
-      // MXFP4: undo the A producer's per-row offsets 2^c_r (rows of acc0 and acc1).
-      // The producer of a unit's rows wrote them before its first k-block,
-      // which precedes acc_full; it cannot be four units ahead of this read.
+      // MXFP4: undo the A producers' per-row offsets 2^c_r (rows of acc0 and
+      // acc1), written before this unit's first stage
       float s0 = 1.f, s1 = 1.f;
       if (AF == kAMxfp4) {
-        s0 = __uint_as_float((uint32_t)(s_crow[un & 3][0][r] + 127) << 23);
-        s1 = __uint_as_float((uint32_t)(s_crow[un & 3][1][r] + 127) << 23);
+        s0 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][0][r] + 127) << 23);
+        s1 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][1][r] + 127) << 23);
       }
       for (int c0 = 0; c0 < n; c0 += 16) {
         uint32_t g[16], h[16];
         tmem_ld16(tbase + lrow + c0, g);
-        tmem_ld16(tbase + lrow + kTcAccCols + c0, h);
+        tmem_ld16(tbase + lrow + args.acc_cols + c0, h);
         tmem_ld_wait();
         if (MODE == 0) {
           const int col = mt * 128 + r;
@@ -524,11 +711,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Activations bf16 -> f16 (n8 groups of 8, 16-byte aligned): exact for
-// |x| in [2^-14, 65504], f16 subnormals below; |x| > 65504 is out of range.
-__global__ void bf16_to_f16_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t n8) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-    const uint4 v = in[i];
+// Activations in pair order for the gate/up GEMM: out[pos] = f16(x[perm[pos] /
+// K]), rows of h8 groups of 8 values.  Exact for |x| in [2^-14, 65504], f16
+// subnormals below; |x| > 65504 is out of range.
+__global__ void gather_f16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int K, int h8,
+                                  int64_t rows, uint4* __restrict__ out) {
+  const int64_t n = rows * h8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / h8;
+    const int c = (int)(i - row * h8);
+    const uint4 v = x[(int64_t)(perm[row] / K) * h8 + c];
     out[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
   }
 }

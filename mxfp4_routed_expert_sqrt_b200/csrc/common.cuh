@@ -24,10 +24,17 @@ __device__ int32_t g_error;
 
 __device__ __forceinline__ void set_error(int32_t code) { atomicCAS(&g_error, 0, code); }
 
-// Upper bound on polls of one mbarrier phase before a kernel gives up
-// (~seconds with the back-off below; a copy that has not landed by then
-// never will).
-constexpr uint32_t kMaxPolls = 1u << 24;
+// Upper bound on the time a kernel waits for one mbarrier phase before it
+// gives up (a copy that has not landed by then never will), and on the number
+// of polls (try_wait itself may suspend the thread for a while).
+constexpr uint64_t kMaxWaitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kMaxPolls = 1u << 26;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,9 +71,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
   for (uint32_t i = 0; i < kMaxPolls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (i >= 32) __nanosleep(64);
+    if (i >= 32) {
+      __nanosleep(64);
+      if ((i & 255) == 0 && global_ns() - t0 > kMaxWaitNs) return false;
+    }
   }
   return false;
 }

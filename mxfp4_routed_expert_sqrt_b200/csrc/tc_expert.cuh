@@ -368,6 +368,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     set_error(kErrWaitTc);
     *reinterpret_cast<volatile int32_t*>(&s_abort) = 1;
   };
+  // bounded wait whose outcome is the same for the whole warp (the tcgen05
+  // loads and stores that follow are taken by whole warps)
+  auto warp_wait = [&](uint64_t* bar, uint32_t ph) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, ph) ? 1 : 0) != 0;
+  };
 
   if (warp >= 4 && warp < 12) {
     // ------------------------------ A producers --------------------------------
@@ -395,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
     auto wait_stage = [&]() -> bool {  // TMEM stage free (its MMAs done)
-      if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) return false;
+      if (!warp_wait(&empty[rs.s], rs.ph ^ 1)) return false;
       tc_fence_after();
       return true;
     };
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if ((int)blockIdx.x < n_units) sc_issue(blockIdx.x, 0);
       cp_async_commit();
       uint32_t un = 0;
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+      for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x, ++un) {
         if (u + (int)gridDim.x < n_units) sc_issue(u + gridDim.x, (un + 1) & 1);
         cp_async_commit();
         cp_async_wait<1>();  // this unit's E8M0 row has landed
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         bool ok = true;
         for (int st = 0; st < nst && ok; ++st) {
-          if (js == 0 && !mbar_wait(&w_full[rw.s], rw.ph)) {
+          if (js == 0 && !warp_wait(&w_full[rw.s], rw.ph)) {
             ok = false;
             break;
           }
@@ -492,10 +497,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v[4 * c + 3] = w.w;
         }
       };
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x) {
         bool ok = true;
         for (int st = 0; st < nst && ok; ++st) {
-          if (!mbar_wait(&w_full[rw.s], rw.ph)) {
+          if (!warp_wait(&w_full[rw.s], rw.ph)) {
             ok = false;
             break;
           }
@@ -651,10 +656,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp;  // TMEM lanes 32q..32q+31
     const int r = q * 32 + lane;
     uint32_t un = 0;
-    for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
+    for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x, ++un) {
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
-      if (!mbar_wait(&acc_full, un & 1)) { give_up(); break; }
+      if (!warp_wait(&acc_full, un & 1)) { give_up(); break; }
       tc_fence_after();
       const uint32_t lrow = (uint32_t)(q * 32) << 16;
       // MXFP4: undo the A producers' per-row offsets 2^c_r (rows of acc0 and

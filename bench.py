@@ -300,12 +300,14 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     assert m.moe_device_error() == 0
 
     def expert_bytes(j, s):
-        # weights of the distinct experts + activations: x read (bf16) and its f16 copy
-        # written and read, h (f16) written and read, y_perm (fp32) written
+        # algorithmic bytes of one moe_expert_gemm call: the weights of the distinct
+        # experts, x read once (bf16), h (f16) written and read between the two
+        # GEMMs, y_perm (fp32) written.  The pair-ordered f16 copy of x the call
+        # makes for its token operand is an implementation detail, not counted.
         B = batches[j][0]
         U = distinct[(j, s)]
         I = dims.inter
-        act = B * H * 2 + 2 * B * H * 2 + 2 * B * K * I * 2 + B * K * H * 4
+        act = B * H * 2 + 2 * B * K * I * 2 + B * K * H * 4
         return U * (3 * (I * H // 2 + I * H // 32)) + act
 
     # route 2 (3 with the tensor-core router split), permute 1, shared 2,

@@ -264,8 +264,9 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
     a.out = logits;
     if ((st = launch_tc<1, kABf16>(xmap, a, s)) != MOE_OK) return st;
   } else {
-    dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
-    route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
+    dim3 g1((E + kLogitExperts - 1) / kLogitExperts, (T + kLogitTokBlock - 1) / kLogitTokBlock);
+    route_logits_kernel<<<g1, kLogitThreads, kLogitExperts * H * sizeof(float), s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
     if ((st = launch_status()) != MOE_OK) return st;
   }
   route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
@@ -290,8 +291,9 @@ moe_status moe_route_noalloc(const moe_dims* dims, const void* x, int32_t T, con
   if (noalloc_scratch(&logits) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int E = dims->n_experts, H = dims->hidden;
-  dim3 g1((E + 3) / 4, (T + kLogitTok - 1) / kLogitTok);
-  route_logits_kernel<<<g1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
+  dim3 g1((E + kLogitExperts - 1) / kLogitExperts, (T + kLogitTokBlock - 1) / kLogitTokBlock);
+  route_logits_kernel<<<g1, kLogitThreads, kLogitExperts * H * sizeof(float), s>>>(
+      static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
   if ((st = launch_status()) != MOE_OK) return st;
   route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
       logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table, vocab,

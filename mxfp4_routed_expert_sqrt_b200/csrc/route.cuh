@@ -13,43 +13,75 @@
 
 namespace moe {
 
-constexpr int kLogitTok = 8;  // tokens per CTA in the SIMT logits kernel
+constexpr int kLogitExperts = 2;     // expert rows per CTA, staged in shared memory
+constexpr int kLogitThreads = 256;
+constexpr int kLogitTokBlock = 64;   // tokens per CTA (grid.y covers the rest)
+constexpr int kLogitTokStep = 4;     // tokens a warp works on at once
 
 // logits[t][e] = sum_h x[t][h] * Wr[e][h], fp32 products and sums.
-// One warp per expert; lanes stride the hidden dim in float4 chunks; a CTA
-// covers 4 experts x kLogitTok tokens, so Wr is read once per token block.
-__global__ void __launch_bounds__(128) route_logits_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           int T, int H,
-                                                           const float* __restrict__ wr, int E,
-                                                           float* __restrict__ logits) {
+// A CTA stages kLogitExperts router rows (fp32) in shared memory with every
+// thread loading in parallel, then its 8 warps stream the x rows (bf16, from
+// L2) of up to kLogitTokBlock tokens, kLogitTokStep tokens per warp at a
+// time, lanes striding the hidden dim in groups of 8 columns.  E/2 CTAs keep
+// every SM busy at any token count, and the router (4 MiB at V4-Flash shape)
+// is read from HBM once per token block.  Shared memory: kLogitExperts * H
+// floats.
+__global__ void __launch_bounds__(kLogitThreads) route_logits_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                     int T, int H,
+                                                                     const float* __restrict__ wr, int E,
+                                                                     float* __restrict__ logits) {
+  extern __shared__ float4 s_w4[];  // [kLogitExperts][H / 4]
+  const int e0 = blockIdx.x * kLogitExperts;
+  const int ne = min(kLogitExperts, E - e0);
+  const int h4 = H / 4, h8 = H / 8;
+  const float4* src = reinterpret_cast<const float4*>(wr + (int64_t)e0 * H);
+  for (int i = threadIdx.x; i < ne * h4; i += kLogitThreads) s_w4[i] = __ldg(src + i);
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 4 + warp;
-  const int t0 = blockIdx.y * kLogitTok;
-  if (e >= E) return;
-  const float4* w4 = reinterpret_cast<const float4*>(wr + (int64_t)e * H);
-  float acc[kLogitTok];
+  const int t_end = min(T, (blockIdx.y + 1) * kLogitTokBlock);
+  for (int t0 = blockIdx.y * kLogitTokBlock + warp * kLogitTokStep; t0 < t_end;
+       t0 += (kLogitThreads / 32) * kLogitTokStep) {
+    float acc[kLogitTokStep][kLogitExperts];
 #pragma unroll
-  for (int i = 0; i < kLogitTok; ++i) acc[i] = 0.f;
-  const int nt = min(kLogitTok, T - t0);
-  for (int j = lane; j < H / 4; j += 32) {
-    const float4 w = __ldg(w4 + j);
+    for (int i = 0; i < kLogitTokStep; ++i)
 #pragma unroll
-    for (int i = 0; i < kLogitTok; ++i) {
-      if (i < nt) {
-        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + (int64_t)(t0 + i) * H) + j);
-        acc[i] = fmaf(__uint_as_float(xv.x << 16), w.x, acc[i]);
-        acc[i] = fmaf(__uint_as_float(xv.x & 0xFFFF0000u), w.y, acc[i]);
-        acc[i] = fmaf(__uint_as_float(xv.y << 16), w.z, acc[i]);
-        acc[i] = fmaf(__uint_as_float(xv.y & 0xFFFF0000u), w.w, acc[i]);
+      for (int e = 0; e < kLogitExperts; ++e) acc[i][e] = 0.f;
+#pragma unroll 4
+    for (int j = lane; j < h8; j += 32) {
+      uint4 xv[kLogitTokStep];
+#pragma unroll
+      for (int i = 0; i < kLogitTokStep; ++i)
+        xv[i] = t0 + i < t_end ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)(t0 + i) * H) + j)
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int e = 0; e < kLogitExperts; ++e) {
+        if (e < ne) {
+          const float4 wa = s_w4[e * h4 + 2 * j], wb = s_w4[e * h4 + 2 * j + 1];
+#pragma unroll
+          for (int i = 0; i < kLogitTokStep; ++i) {
+            float a = acc[i][e];
+            a = fmaf(__uint_as_float(xv[i].x << 16), wa.x, a);
+            a = fmaf(__uint_as_float(xv[i].x & 0xFFFF0000u), wa.y, a);
+            a = fmaf(__uint_as_float(xv[i].y << 16), wa.z, a);
+            a = fmaf(__uint_as_float(xv[i].y & 0xFFFF0000u), wa.w, a);
+            a = fmaf(__uint_as_float(xv[i].z << 16), wb.x, a);
+            a = fmaf(__uint_as_float(xv[i].z & 0xFFFF0000u), wb.y, a);
+            a = fmaf(__uint_as_float(xv[i].w << 16), wb.z, a);
+            a = fmaf(__uint_as_float(xv[i].w & 0xFFFF0000u), wb.w, a);
+            acc[i][e] = a;
+          }
+        }
       }
     }
-  }
 #pragma unroll
-  for (int i = 0; i < kLogitTok; ++i) {
-    float v = acc[i];
+    for (int i = 0; i < kLogitTokStep; ++i)
 #pragma unroll
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && i < nt) logits[(int64_t)(t0 + i) * E + e] = v;
+      for (int e = 0; e < kLogitExperts; ++e) {
+        float v = acc[i][e];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && e < ne && t0 + i < t_end) logits[(int64_t)(t0 + i) * E + e0 + e] = v;
+      }
   }
 }
 

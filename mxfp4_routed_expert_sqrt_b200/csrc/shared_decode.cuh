@@ -21,6 +21,7 @@ namespace moe {
 constexpr int kShThreads = 256;
 constexpr int kShWarps = kShThreads / 32;
 constexpr int kShMaxNt = 8;  // token tiles of 8 (T <= 64)
+constexpr int kShBatch = 8;  // column groups whose weights are loaded together
 
 struct ShArgs {
   const __nv_bfloat16* w0;  // MODE 0: gate [I][H]; MODE 1: down [H][I]
@@ -73,17 +74,28 @@ __global__ void __launch_bounds__(kShThreads) shared_decode_kernel(const ShArgs 
 #pragma unroll
   for (int nt = 0; nt < kShMaxNt; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 
-#pragma unroll 2
-  for (int gi = 0; gi < NG; ++gi) {
-    const int G = G0 + gi, GA = G % a_groups;
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(rg + GA * 32 + 8 * t));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(rg8 + GA * 32 + 8 * t));
+  // The weight fragments of kShBatch column groups are loaded before any of
+  // their MMAs, so each warp keeps 2 * kShBatch 16-byte HBM loads in flight.
+  for (int gi0 = 0; gi0 < NG; gi0 += kShBatch) {
+    uint4 a[kShBatch], b[kShBatch];
 #pragma unroll
-    for (int nt = 0; nt < kShMaxNt; ++nt) {
-      if (nt < ntiles) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[nt] + G * 32 + 8 * t));
-        mma_bf16_16816(acc[nt], a.x, b.x, a.y, b.y, xv.x, xv.y);
-        mma_bf16_16816(acc[nt], a.z, b.z, a.w, b.w, xv.z, xv.w);
+    for (int u = 0; u < kShBatch; ++u) {
+      const int GA = (G0 + min(gi0 + u, NG - 1)) % a_groups;
+      a[u] = __ldg(reinterpret_cast<const uint4*>(rg + GA * 32 + 8 * t));
+      b[u] = __ldg(reinterpret_cast<const uint4*>(rg8 + GA * 32 + 8 * t));
+    }
+#pragma unroll
+    for (int u = 0; u < kShBatch; ++u) {
+      if (gi0 + u < NG) {
+        const int G = G0 + gi0 + u;
+#pragma unroll
+        for (int nt = 0; nt < kShMaxNt; ++nt) {
+          if (nt < ntiles) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[nt] + G * 32 + 8 * t));
+            mma_bf16_16816(acc[nt], a[u].x, b[u].x, a[u].y, b[u].y, xv.x, xv.y);
+            mma_bf16_16816(acc[nt], a[u].z, b[u].z, a[u].w, b[u].w, xv.z, xv.w);
+          }
+        }
       }
     }
   }

@@ -104,12 +104,12 @@ bool make_weight_map(CUtensorMap* map, const uint8_t* base, int af, const TcArgs
 }
 
 // Plans the pipeline of one tensor-core expert launch, builds its weight
-// tensor maps and launches it (one CTA per SM).
-template <int MODE, int AF>
-moe_status launch_tc(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
+// tensor maps and launches it (one CTA per SM); EPI epilogue warps.
+template <int MODE, int AF, int EPI>
+moe_status launch_tc_epi(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kTcSmemMax) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured = true;
@@ -122,8 +122,14 @@ moe_status launch_tc(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
   } else {
     w1 = w0;
   }
-  tc_expert_kernel<MODE, AF><<<sm_count(), kTcThreads, a.smem_bytes, s>>>(bmap, w0, w1, a);
+  tc_expert_kernel<MODE, AF, EPI><<<sm_count(), tc_threads(EPI), a.smem_bytes, s>>>(bmap, w0, w1, a);
   return launch_status();
+}
+
+// 128-token chunks get 8 epilogue warps, smaller ones 4.
+template <int MODE, int AF>
+moe_status launch_tc(const CUtensorMap& bmap, const TcArgs& a, cudaStream_t s) {
+  return a.n_chunk > 64 ? launch_tc_epi<MODE, AF, 8>(bmap, a, s) : launch_tc_epi<MODE, AF, 4>(bmap, a, s);
 }
 
 // Tokens per expert-kernel unit: the accumulator columns a unit reserves.  A

@@ -30,9 +30,14 @@
 // cycles that do not overlap the MMAs, so stages are made as long as TMEM
 // allows.
 //
-// Roles (480 threads, one CTA per SM, persistent over units):
-//   warps 0-3   epilogue: tcgen05.ld of the two accumulators (TMEM lane
-//               quadrant = warp), SwiGLU or copy, global stores;
+// Roles (480 or 608 threads, one CTA per SM, persistent over units):
+//   warps 0-3 (and 15-18 when EPI = 8)  epilogue: tcgen05.ld of the two
+//               accumulators (TMEM lane quadrant = warp mod 4; with 8 warps
+//               the two warps of a quadrant take alternate 16-column chunks,
+//               so a wide accumulator is released twice as soon), SwiGLU or
+//               copy, global stores.  8 epilogue warps pay off for 128-token
+//               chunks (prefill); for small chunks the 480-thread launch
+//               leaves the A producers more registers;
 //   warps 4-11  A producers: thread = one weight row of one of the two tiles;
 //               reads its row's bytes from the weight ring (conflict-free: the
 //               ring holds swizzled TMA boxes), converts them exactly and writes
@@ -54,7 +59,8 @@
 
 namespace moe {
 
-constexpr int kTcThreads = 480;
+// Threads of a launch with EPI epilogue warps (4: warps 0-3; 8: also 15-18).
+__host__ __device__ constexpr int tc_threads(int epi) { return (11 + epi) * 32; }
 constexpr int kTcKB = 64;      // k per k-block (one 128-byte swizzle atom of 16-bit values)
 constexpr int kTcKG = 2;       // k-blocks per pipeline stage
 constexpr int kTcStageK = kTcKB * kTcKG;
@@ -273,8 +279,8 @@ inline bool tc_plan(TcArgs& a, int af) {
   return a.smem_bytes <= kTcSmemMax;
 }
 
-template <int MODE, int AF>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int MODE, int AF, int EPI>
+__global__ void __launch_bounds__(tc_threads(EPI), 1)
     tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap0,
                      const __grid_constant__ CUtensorMap wmap1, const TcArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&w_empty[s], 8);
     }
     mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, 4);
+    mbar_init(&acc_empty, EPI);
     mbar_init(&mma_done, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -648,12 +654,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&mma_done, 0)) set_error(kErrWaitTc);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 4 || (EPI == 8 && warp >= 15)) {
     // ------------------------------ epilogue ----------------------------------
     // MODE 0, MXFP4: h = swiglu(gate, up) in f16 [pos][rows]
     // MODE 0, bf16:  h as a bf16 pair, hi at [pos][col], lo = h - hi at [pos][rows + col]
     // MODE 1:        fp32 [pos][rows], both row tiles
-    const int q = warp;  // TMEM lanes 32q..32q+31
+    const int q = warp & 3;             // TMEM lanes 32q..32q+31
+    const int half = warp >= 15 ? 1 : 0;  // EPI = 8: the two warps of a quadrant take alternate 16-column chunks
     const int r = q * 32 + lane;
     uint32_t un = 0;
     for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x, ++un) {
@@ -669,7 +676,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         s0 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][0][r] + 127) << 23);
         s1 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][1][r] + 127) << 23);
       }
-      for (int c0 = 0; c0 < n; c0 += 16) {
+      for (int c0 = 16 * half; c0 < n; c0 += 16 * (EPI / 4)) {
         uint32_t g[16], h[16];
         tmem_ld16(tbase + lrow + c0, g);
         tmem_ld16(tbase + lrow + args.acc_cols + c0, h);

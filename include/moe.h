@@ -90,8 +90,18 @@ const char* moe_status_string(moe_status status);
 
 /* Reads and clears the device error word of the current device (host call,
  * synchronises the current device).  0 = no error; otherwise a code naming
- * the kernel that gave up a bounded wait. */
+ * the kernel that gave up a bounded wait: 0x201 an expert id outside [0, E)
+ * reached moe_permute, 0x301 a tensor-core kernel gave up waiting on a copy
+ * (each wait is bounded to 2 s), 0x401 moe_selftest_wait. */
 int32_t moe_device_error(void);
+
+/* Health check of the bounded-wait path (no counterpart on the pages): a
+ * kernel waits on a barrier that nothing releases, gives up after wait_us
+ * microseconds (1 .. 2,000,000), records device error 0x401 and returns,
+ * exactly as the pipeline kernels do when a copy never lands.  Afterwards
+ * moe_device_error() returns 0x401 and the device stays usable.  Enqueued on
+ * `stream`; returns MOE_ERR_INVALID_ARG for a wait outside the range. */
+moe_status moe_selftest_wait(int32_t wait_us, void* stream);
 
 /* --- routing ---------------------------------------------------------- */
 

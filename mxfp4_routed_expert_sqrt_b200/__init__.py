@@ -19,7 +19,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3
                 4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_DEVICE"}
 
 # every symbol include/moe.h declares
-EXPORTS = ("moe_abi_version", "moe_status_string", "moe_device_error", "moe_route_workspace_size",
+EXPORTS = ("moe_abi_version", "moe_status_string", "moe_device_error", "moe_selftest_wait",
+           "moe_route_workspace_size",
            "moe_route", "moe_route_noalloc", "moe_permute_workspace_size", "moe_permute",
            "moe_expert_gemm_workspace_size", "moe_expert_gemm", "shared_expert_workspace_size",
            "shared_expert", "moe_combine")
@@ -61,6 +62,8 @@ def lib():
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_device_error.restype = ctypes.c_int32
         L.moe_device_error.argtypes = []
+        L.moe_selftest_wait.restype = ctypes.c_int
+        L.moe_selftest_wait.argtypes = [_i32, _vp]
         L.moe_route_workspace_size.restype = _sz
         L.moe_route_workspace_size.argtypes = [dp, _i32]
         L.moe_route.restype = ctypes.c_int
@@ -131,6 +134,18 @@ def moe_abi_version() -> int:
 
 def moe_device_error() -> int:
     return lib().moe_device_error()
+
+
+# device error codes (moe_device_error)
+DEVICE_ERR_BAD_EXPERT = 0x201
+DEVICE_ERR_WAIT_TC = 0x301
+DEVICE_ERR_WAIT_SELFTEST = 0x401
+
+
+def moe_selftest_wait(wait_us: int, stream=None):
+    """Enqueues the bounded-wait health check: a kernel that waits on a barrier
+    nothing releases, gives up after wait_us and records device error 0x401."""
+    _check("moe_selftest_wait", lib().moe_selftest_wait(wait_us, _stream(stream)))
 
 
 def moe_route_workspace_size(dims, T) -> int:

@@ -15,9 +15,9 @@ namespace moe {
 // Device error codes written to g_error (first writer wins).
 enum : int32_t {
   kErrNone = 0,
-  kErrWaitDecode = 0x101,   // decode expert kernel gave up waiting for a bulk copy
   kErrBadExpert = 0x201,    // an expert id outside [0, E) reached moe_permute
   kErrWaitTc = 0x301,       // tensor-core kernel gave up waiting on an mbarrier
+  kErrWaitSelftest = 0x401, // moe_selftest_wait: its wait ran out, as it should
 };
 
 __device__ int32_t g_error;
@@ -69,18 +69,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity to complete: false after
+// max_ns of %globaltimer time (or kMaxPolls polls).
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t max_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 0; i < kMaxPolls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (i >= 32) {
       __nanosleep(64);
-      if ((i & 255) == 0 && global_ns() - t0 > kMaxWaitNs) return false;
+      if ((i & 255) == 0 && global_ns() - t0 > max_ns) return false;
     }
   }
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_ns(bar, parity, kMaxWaitNs);
+}
+
+// The bounded-wait path on its own: waits for a phase of a fresh mbarrier
+// that nothing arrives on, gives up after max_ns, records kErrWaitSelftest
+// and returns (what every pipeline kernel does when a copy never lands).
+__global__ void selftest_wait_kernel(uint64_t max_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_ns(&bar, 0, max_ns)) set_error(kErrWaitSelftest);
+  }
 }
 
 // 1-D bulk copy global -> shared (async proxy), completion counted in bytes

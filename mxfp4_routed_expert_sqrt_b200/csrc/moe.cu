@@ -227,6 +227,12 @@ int32_t moe_device_error(void) {
   return v;
 }
 
+moe_status moe_selftest_wait(int32_t wait_us, void* stream) {
+  if (wait_us <= 0 || wait_us > 2000000) return MOE_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)wait_us * 1000u);
+  return launch_status();
+}
+
 size_t moe_route_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
   size_t b = round_up((size_t)T * dims->n_experts * sizeof(float), 256);

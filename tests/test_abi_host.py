@@ -89,6 +89,13 @@ def test_argument_errors_return_before_launch(m):
                       None, None, None, None, 0, 0)
 
 
+def test_selftest_wait_rejects_out_of_range_waits(m):
+    for bad in (0, -5, 2_000_001):
+        with pytest.raises(m.MoeError) as e:
+            m.moe_selftest_wait(bad, 0)
+        assert e.value.status == 1
+
+
 def test_projection_validation(m):
     d = gen.V4
     fake = 1 << 40

@@ -267,7 +267,7 @@ inline bool tc_plan(TcArgs& a, int af) {
   const int bst = kTcKG * nc * 128;
   const int sc = af == kAMxfp4 ? 2 * kTcAThreads * a.sr : 0;
   const int groups = a.offsets != nullptr ? a.E : 1;
-  const int pre = ((groups + 1) * 4 + 127) / 128 * 128;
+  const int pre = (2 * (groups + 1) * 4 + 127) / 128 * 128;  // unit prefix + group offsets
   const int budget = kTcSmemMax - 1024;  // 1024: alignment slack of the dynamic base
   const int w = (budget - a.stages * bst - sc - pre) / a.w_slot_bytes;
   a.w_slots = w < 6 ? w : 6;
@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   uint8_t* s_w = smem;                  // weight ring
   uint8_t* s_b = smem + args.off_b;     // token tiles, one per stage
   uint8_t* s_sc = smem + args.off_sc;   // E8M0 rows, two unit buffers, thread-major
-  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + args.off_prefix);  // [E + 1]
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + args.off_prefix);  // [E + 1] units before group e
+  int32_t* s_off = s_prefix + (args.offsets != nullptr ? args.E : 1) + 1;  // [E + 1] copy of offsets
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool grouped = args.offsets != nullptr;
@@ -309,13 +310,18 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   const uint32_t a_base = 2 * args.acc_cols;
 
   // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
+  // The group offsets are read once, by all threads in parallel, into shared
+  // memory: the scan and every unit lookup then stay on chip.
+  if (grouped)
+    for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
+  __syncthreads();
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
       int c = 0;
       if (e < E) {
-        const int n = grouped ? args.offsets[e + 1] - args.offsets[e] : args.n_single;
+        const int n = grouped ? s_off[e + 1] - s_off[e] : args.n_single;
         c = MT * ((n + NC - 1) / NC);
       }
       int incl = c;
@@ -364,8 +370,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     const int local = u - s_prefix[e];
     mt = local % MT;
     const int chunk = local / MT;
-    const int start = grouped ? args.offsets[e] : 0;
-    const int ne = grouped ? args.offsets[e + 1] - start : args.n_single;
+    const int start = grouped ? s_off[e] : 0;
+    const int ne = grouped ? s_off[e + 1] - start : args.n_single;
     pos0 = start + chunk * NC;
     n = min(NC, ne - chunk * NC);
   };

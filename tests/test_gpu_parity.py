@@ -156,21 +156,33 @@ def _expert_gemm(dc, T):
     return idx, perm.cpu().numpy()[:T * K], y[:T * K * H].view(T * K, H).cpu().numpy()
 
 
-# T <= 64 runs the decode path, larger T the tensor-core grouped GEMM
-EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64), ("tiny_T37", gen.TINY, 37, 74), ("v4_T1", gen.V4, 1, 6),
-                ("v4_T8", gen.V4, 8, 48), ("v4_T37", gen.V4, 37, 24), ("v4_T64", gen.V4, 64, 24),
-                ("tiny_T100_tc", gen.TINY, 100, 200), ("tiny_T1000_tc", gen.TINY, 1000, 120),
-                ("v4_T96_tc", gen.V4, 96, 24), ("v4_T300_tc", gen.V4, 300, 24)]
+# The call picks its token chunk (32, 64 or 128 pairs per unit) from the mean
+# pairs per expert; the zipf case piles most pairs onto a few experts, so their
+# groups span many 32-pair chunks, and it samples both sides of every chunk
+# boundary of the most loaded expert.
+EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64, None), ("tiny_T37", gen.TINY, 37, 74, None),
+                ("v4_T1", gen.V4, 1, 6, None), ("v4_T8", gen.V4, 8, 48, None), ("v4_T37", gen.V4, 37, 24, None),
+                ("v4_T64", gen.V4, 64, 24, None), ("tiny_T100_tc", gen.TINY, 100, 200, None),
+                ("tiny_T1000_tc", gen.TINY, 1000, 120, None), ("v4_T96_tc", gen.V4, 96, 24, None),
+                ("v4_T300_tc", gen.V4, 300, 24, None), ("v4_zipf_T256_chunks", gen.V4, 256, 16, "zipf")]
 
 
-@pytest.mark.parametrize("name,dims,T,nsample", EXPERT_CASES, ids=[c[0] for c in EXPERT_CASES])
-def test_expert_gemm_parity(name, dims, T, nsample):
-    c = make_case(dims, T, with_shared=False)
+@pytest.mark.parametrize("name,dims,T,nsample,bias", EXPERT_CASES, ids=[c[0] for c in EXPERT_CASES])
+def test_expert_gemm_parity(name, dims, T, nsample, bias):
+    c = make_case(dims, T, with_shared=False, bias=_zipf_bias() if bias == "zipf" else None)
     dc = DeviceCase(c, DEV)
     idx, perm, y = _expert_gemm(dc, T)
     K = dims.top_k
     rng = np.random.default_rng(1)
-    positions = np.sort(rng.choice(T * K, size=min(nsample, T * K), replace=False))
+    positions = rng.choice(T * K, size=min(nsample, T * K), replace=False)
+    if bias == "zipf":
+        counts = np.bincount(idx.reshape(-1), minlength=dims.n_experts)
+        hot = int(np.argmax(counts))
+        assert counts[hot] > 2 * 32, f"{name}: the most loaded expert has only {counts[hot]} pairs"
+        start = int(counts[:hot].sum())
+        edges = [j for b in range(32, int(counts[hot]), 32) for j in (b - 1, b)] + [0, int(counts[hot]) - 1]
+        positions = np.concatenate([positions, start + np.array(edges)])
+    positions = np.unique(positions)
     xs_all = (c.x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     got, want = [], []
     for pos in positions:

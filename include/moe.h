@@ -193,9 +193,15 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *           is f16.
  *  offsets, perm  as written by moe_permute.
  *  y_perm   fp32 [T*top_k][hidden] out.
- *  ws       device workspace of moe_expert_gemm_workspace_size() bytes.
- * One grouped tcgen05 GEMM pair for every T; the number of units follows the
- * device-side counts, the launch does not depend on them.
+ *  ws       device workspace of moe_expert_gemm_workspace_size() bytes: the
+ *           pairs' activations in expert order as f16 [T*top_k][hidden], then
+ *           h in f16 [T*top_k][inter].
+ * Shapes: inter a multiple of 128, hidden a multiple of 256 (the row tiles of
+ * the two GEMMs), besides the moe_dims limits; other shapes return
+ * MOE_ERR_UNSUPPORTED before anything is enqueued.
+ * One grouped tcgen05 GEMM pair for every T (plus the activation gather); the
+ * number of units follows the device-side counts, the launches do not depend
+ * on them.  A kernel that gives up a bounded wait records device error 0x301.
  */
 moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
                            moe_mxfp4_proj up, moe_mxfp4_proj down, const int32_t* offsets,

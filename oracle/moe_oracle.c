@@ -30,7 +30,7 @@
  *  [JANG]    "DeepSeek-V4-Flash-0731-JANG", Dynamic affine recipe table: the
  *            router is kept in f32 (its weight is an fp32 input here).
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent (each one a choice of this oracle):
  *  - nibble order: the low nibble of a byte is the even column;
  *  - blob order: nibble plane [rows][cols/2], then scale plane [rows][cols/32];
  *  - the scale group is 32 consecutive input columns of one output row;

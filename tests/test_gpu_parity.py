@@ -252,12 +252,17 @@ LAYER_CASES = [("tiny_T8", gen.TINY, 8, None, False, 8), ("tiny_T1", gen.TINY, 1
                ("v4_zipf_T32_layer0", gen.V4, 32, "zipf", False, 8),
                ("v4_decode_T1", gen.V4, 1, None, False, 1), ("v4_decode_T8", gen.V4, 8, None, False, 8),
                ("v4_decode_T32", gen.V4, 32, None, False, 8), ("v4_decode_T64", gen.V4, 64, None, False, 8),
-               ("v4_hash_T2048", gen.V4, 2048, None, True, 6), ("v4_prefill_T4096", gen.V4, 4096, None, False, 6)]
+               ("v4_hash_T2048", gen.V4, 2048, None, True, 6), ("v4_prefill_T4096", gen.V4, 4096, None, False, 6),
+               # degenerate routing: every table row names the same 6 experts, so all
+               # 1,800 pairs land on them (ten 32-pair chunks each) and 250 experts are empty
+               ("v4_hash_all_same_T300", gen.V4, 300, None, "same", 6)]
 
 
 @pytest.mark.parametrize("name,dims,T,bias,hashed,nsample", LAYER_CASES, ids=[c[0] for c in LAYER_CASES])
 def test_layer_parity(name, dims, T, bias, hashed, nsample):
-    c = make_case(dims, T, hashed=hashed, bias=_zipf_bias() if bias == "zipf" else None)
+    c = make_case(dims, T, hashed=bool(hashed), bias=_zipf_bias() if bias == "zipf" else None)
+    if hashed == "same":
+        c.table = np.ascontiguousarray(np.broadcast_to(c.table[0], c.table.shape))
     dc = DeviceCase(c, DEV)
     layer = m.MoeLayer(dims, T, DEV)
     out = _f32(T * dims.hidden)

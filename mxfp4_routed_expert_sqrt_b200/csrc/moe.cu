@@ -1,5 +1,6 @@
 // libmoe.so: the C ABI declared in include/moe.h.  One translation unit: the
 // kernels live in the headers included below.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -22,6 +23,20 @@ int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
+}
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once
+// per device (the attribute belongs to each device's context); `done` holds
+// one bit per device id.
+template <class Kernel>
+bool smem_limit_once(std::atomic<uint64_t>& done, Kernel* kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit, std::memory_order_release);
+  return true;
 }
 
 moe_status launch_status() {
@@ -107,13 +122,8 @@ bool make_weight_map(CUtensorMap* map, const uint8_t* base, int af, const TcArgs
 // tensor maps and launches it (one CTA per SM); EPI epilogue warps.
 template <int MODE, int AF, int EPI>
 moe_status launch_tc_epi(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(tc_expert_kernel<MODE, AF, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kTcSmemMax) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (!smem_limit_once(configured, tc_expert_kernel<MODE, AF, EPI>, kTcSmemMax)) return MOE_ERR_CUDA;
   if (!tc_plan(a, AF)) return MOE_ERR_UNSUPPORTED;
   CUtensorMap w0, w1;
   if (!make_weight_map(&w0, a.w0, AF, a)) return MOE_ERR_CUDA;
@@ -326,13 +336,8 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
   if (!offsets || (T > 0 && (!topk_idx || !perm || !inv))) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int smem = 32 * E * (int)sizeof(int32_t);
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * 4) !=
-        cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (!smem_limit_once(configured, permute_kernel, 32 * 1024 * 4)) return MOE_ERR_CUDA;
   permute_kernel<<<1, kPermuteThreads, smem, s>>>(topk_idx, T * K, E, offsets, perm, inv);
   return launch_status();
 }

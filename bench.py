@@ -237,6 +237,22 @@ def traffic_record(desc):
     return rec.get("bytes_per_launch")
 
 
+def max_over_ranks(dist, value, device):
+    """The maximum of `value` over all ranks; the rank's own value without a
+    process group (one GPU)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_step_per_rank, steps, seconds):
+    """Units all ranks processed per second of the slowest rank."""
+    return world * units_per_step_per_rank * steps / seconds
+
+
 def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     import torch
 
@@ -384,13 +400,9 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         warm_graph.replay()
         torch.cuda.synchronize()
     sampler.stop()
-    ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(dist, ev0.elapsed_time(ev1), dev)
     tokens_per_step = sum(B for B, _ in batches)
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, args.steps, ms / 1e3)
 
     # roofline of the routed-expert GEMV (moe_expert_gemm: gate/up and down launches)
     k_ms, k_bytes, n_calls = 0.0, 0, 0
@@ -447,18 +459,18 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    e0 = time.perf_counter()
+    # device-timed on the replay stream; each step waits for its result on the
+    # host, so the region holds the copies, the layer and the host round trip
+    ev_e0, ev_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_e0.record(stream)
     for _ in range(args.steps):
         for ge in graphs_e2e:
             ge()
         stream.synchronize()
-    e1 = time.perf_counter()
-    e2e_s = e1 - e0
-    if dist is not None:
-        tt = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
-    e2e = {"value": world * tokens_per_step * args.steps / e2e_s, "unit": unit,
+    ev_e1.record(stream)
+    ev_e1.synchronize()
+    e2e_s = max_over_ranks(dist, ev_e0.elapsed_time(ev_e1) / 1e3, dev)
+    e2e = {"value": whole_job_rate(world, tokens_per_step, args.steps, e2e_s), "unit": unit,
            "h2d_bytes_per_step": sum(B * H * 2 for B, _ in batches),
            "d2h_bytes_per_step": sum(B * H * 4 for B, _ in batches)}
     assert m.moe_device_error() == 0

@@ -420,9 +420,11 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         peaks = _json.load(open(pk))
     traffic = traffic_record(desc)
     kernel = "tc_expert_kernel (moe_expert_gemm: gate/up+SwiGLU and down, tcgen05)"
-    if args.workload in ("prefill", "hash"):
-        # tensor bound: algorithmic flops = pairs * 3 projections * 2 * H * I (f16 x f16,
-        # same nominal rate as bf16); the GEMM runs inside a multi-millisecond step
+    if args.workload == "prefill":
+        # tensor bound (~96 pairs per expert, arithmetic intensity above the ridge):
+        # algorithmic flops = pairs * 3 projections * 2 * H * I (f16 x f16, same
+        # nominal rate as bf16); the GEMM runs inside a multi-millisecond step.
+        # The hash workload (~48 pairs per expert) sits below the ridge: HBM bound.
         flops = sum(B * K * 3 * 2 * H * dims.inter for B, _ in batches) * args.steps
         peak = peaks.get("bf16_tflops_sustained")
         peak_src = "measured sustained bf16" if peak else "fallback sustained"

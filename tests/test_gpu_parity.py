@@ -117,13 +117,19 @@ def test_route_parity(name, dims, T, bias, hashed):
 
 # ---- grouping --------------------------------------------------------------------
 
+# the largest calls moe_permute accepts: T*K up to 2^22 pairs, E up to 1024, K up to 32
 @pytest.mark.parametrize("T,K,E,mode", [(0, 6, 256, "rand"), (1, 6, 256, "rand"), (64, 6, 256, "rand"),
                                         (4096, 6, 256, "rand"), (37, 2, 16, "rand"),
-                                        (1000, 6, 256, "one_hot"), (2048, 6, 256, "skew")])
+                                        (1000, 6, 256, "one_hot"), (2048, 6, 256, "skew"),
+                                        (699050, 6, 256, "stride"), (131072, 32, 1024, "stride")])
 def test_permute_parity(T, K, E, mode):
     rng = np.random.default_rng(T + E)
     if mode == "rand":
         idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]) if T else np.zeros((0, K))
+    elif mode == "stride":  # K distinct ids per token: (r + k * s) mod E, s odd, E a power of two
+        r = rng.integers(0, E, size=(T, 1))
+        st = 2 * rng.integers(0, E // 2, size=(T, 1)) + 1
+        idx = (r + np.arange(K)[None, :] * st) % E
     elif mode == "one_hot":  # every token picks the same K experts
         idx = np.tile(np.arange(K), (T, 1))
     else:  # Zipf-like popularity
@@ -136,6 +142,22 @@ def test_permute_parity(T, K, E, mode):
     assert np.array_equal(off, roff)
     assert np.array_equal(perm, rperm)
     assert np.array_equal(inv, rinv)
+
+
+def test_permute_reports_an_expert_id_out_of_range():
+    # the kernel's own bounds check: the bad ids count as expert 0 and device
+    # error 0x201 is recorded; every write stays inside the output buffers
+    T, K, E = 64, 6, 256
+    rng = np.random.default_rng(7)
+    idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    idx[3, 2] = E
+    idx[40, 5] = -1
+    assert m.moe_device_error() == 0
+    off, perm, inv = run_permute(torch.from_numpy(idx.reshape(-1).copy()).to(DEV), T, K, E)
+    assert m.moe_device_error() == m.DEVICE_ERR_BAD_EXPERT
+    assert np.array_equal(np.sort(perm), np.arange(T * K))
+    assert np.array_equal(inv[perm], np.arange(T * K))
+    assert off[E] == T * K
 
 
 # ---- experts, shared, combine -------------------------------------------------------

@@ -220,19 +220,34 @@ def run_reference(args, dims, batches, desc, metric, unit):
 # the CUDA path
 # ---------------------------------------------------------------------------------------
 
-def kernel_source_hash():
+# moe_expert_gemm runs the block-scaled kernel when an expert averages at most
+# 8 pairs (the library's path choice from T), else the dequantising kernel.
+EXPERT_KERNELS = {
+    "block_scaled": ("mx_expert_kernel (moe_expert_gemm: block-scaled tcgen05 mxf8f6f4, gate/up+SwiGLU and down)",
+                     ("mx_expert.cuh", "tc_expert.cuh", "common.cuh")),
+    "dequant": ("tc_expert_kernel (moe_expert_gemm: E2M1 dequantised to f16, tcgen05 f16, gate/up+SwiGLU and down)",
+                ("tc_expert.cuh", "common.cuh")),
+}
+
+
+def expert_path(dims, B):
+    avg = -(-B * dims.top_k // dims.n_experts)
+    return "block_scaled" if avg <= 8 else "dequant"
+
+
+def kernel_source_hash(path):
     h = hashlib.sha256()
-    for f in ("tc_expert.cuh", "common.cuh"):
+    for f in EXPERT_KERNELS[path][1]:
         h.update(open(os.path.join(ROOT, "mxfp4_routed_expert_sqrt_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def traffic_record(desc):
+def traffic_record(desc, path):
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p)).get(desc)
-    if not rec or rec.get("kernel_hash") != kernel_source_hash():
+    if not rec or rec.get("kernel_hash") != kernel_source_hash(path):
         return None
     return rec.get("bytes_per_launch")
 
@@ -317,9 +332,10 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
 
     def expert_bytes(j, s):
         # algorithmic bytes of one moe_expert_gemm call: the weights of the distinct
-        # experts, x read once (bf16), h (f16) written and read between the two
-        # GEMMs, y_perm (fp32) written.  The pair-ordered f16 copy of x the call
-        # makes for its token operand is an implementation detail, not counted.
+        # experts, x read once (bf16), h written and read between the two GEMMs
+        # (counted at 2 bytes a value), y_perm (fp32) written.  The pair-ordered
+        # copy of x the call makes for its token operand (E4M3 terms or f16) is an
+        # implementation detail, not counted.
         B = batches[j][0]
         U = distinct[(j, s)]
         I = dims.inter
@@ -327,7 +343,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         return U * (3 * (I * H // 2 + I * H // 32)) + act
 
     # route 2 (3 with the tensor-core router split), permute 1, shared 2,
-    # experts 3 (x to f16, gate/up, down), combine 1
+    # experts 3 (activation gather, gate/up, down), combine 1
     n_layer_kernels = 9 + (1 if batches[0][0] > 64 and dims.n_experts % 256 == 0 else 0)
 
     def one_step(i, events=None):
@@ -418,8 +434,10 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk):
         peaks = _json.load(open(pk))
-    traffic = traffic_record(desc)
-    kernel = "tc_expert_kernel (moe_expert_gemm: gate/up+SwiGLU and down, tcgen05)"
+    path = expert_path(dims, batches[0][0])
+    assert all(expert_path(dims, B) == path for B, _ in batches)
+    traffic = traffic_record(desc, path)
+    kernel = EXPERT_KERNELS[path][0]
     if args.workload == "prefill":
         # tensor bound (~96 pairs per expert, arithmetic intensity above the ridge):
         # algorithmic flops = pairs * 3 projections * 2 * H * I (f16 x f16, same
@@ -519,7 +537,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("mine", "reference"), default="mine")
     ap.add_argument("--workload", default="decode", choices=("decode", "decode64", "prefill", "hash", "stack8", "tiny"))

@@ -182,24 +182,33 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  * All routed experts for the grouped pairs:
  *   y_perm[pos] = Wd_e (silu(min(Wg_e x_t, L)) * clamp(Wu_e x_t, -L, L))
  * for pos in [offsets[e], offsets[e+1]), p = perm[pos], t = p / top_k.
- *  x        bf16 [T][hidden], 16-byte aligned; converted to f16 on the way
- *           in, so |x| must stay below 65504 (values under 2^-14 keep f16
- *           subnormal precision).
+ *  x        bf16 [T][hidden], 16-byte aligned.
  *  gate, up MXFP4 [inter][hidden]; down MXFP4 [hidden][inter] (see
- *           moe_mxfp4_proj).  Every weight is dequantised exactly (to f16, up
- *           to a power of two per row undone in fp32) as long as the E8M0
- *           exponents of one weight row span at most 36 octaves; products are
- *           exact and sums fp32 on the tensor cores.  h between the two GEMMs
- *           is f16.
+ *           moe_mxfp4_proj).
  *  offsets, perm  as written by moe_permute.
  *  y_perm   fp32 [T*top_k][hidden] out.
- *  ws       device workspace of moe_expert_gemm_workspace_size() bytes: the
- *           pairs' activations in expert order as f16 [T*top_k][hidden], then
- *           h in f16 [T*top_k][inter].
+ *  ws       device workspace of moe_expert_gemm_workspace_size(dims, T)
+ *           bytes (its layout depends on the path below).
+ * Two paths, chosen from T alone (mean pairs per expert, ceil(T*top_k / E)):
+ *  - at most 8 (decode): block-scaled tensor-core MMAs
+ *    (tcgen05 kind::mxf8f6f4): the E2M1 codes and E8M0 scales go to the
+ *    tensor core as stored and are applied there.  Each activation enters as
+ *    two E4M3 terms with E8M0 group-32 scales (a bf16 x is carried exactly
+ *    unless a residual falls below the E4M3 range of its 32-value group), h
+ *    between the GEMMs as three terms (about 12 significant bits); sums fp32.
+ *    Workspace: E4M3 terms and E8M0 scales of x in expert order
+ *    [2][T*top_k][hidden] and [2][T*top_k][hidden/32], then of h
+ *    [3][T*top_k][inter] and [3][T*top_k][inter/32] bytes.
+ *  - above 8 (prefill): each weight is dequantised exactly to f16 (up to a
+ *    power of two per row undone in fp32) as long as the E8M0 exponents of
+ *    one weight row span at most 36 octaves; x goes in as f16 (|x| below
+ *    65504, values under 2^-14 keep f16 subnormal precision), h between the
+ *    GEMMs is f16; f16 x f16 MMAs with fp32 sums.  Workspace: x in expert
+ *    order as f16 [T*top_k][hidden], then h in f16 [T*top_k][inter].
  * Shapes: inter a multiple of 128, hidden a multiple of 256 (the row tiles of
  * the two GEMMs), besides the moe_dims limits; other shapes return
  * MOE_ERR_UNSUPPORTED before anything is enqueued.
- * One grouped tcgen05 GEMM pair for every T (plus the activation gather); the
+ * Either path is one grouped tcgen05 GEMM pair plus the activation gather; the
  * number of units follows the device-side counts, the launches do not depend
  * on them.  A kernel that gives up a bounded wait records device error 0x301.
  */

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "mx_expert.cuh"
 #include "tc_expert.cuh"
 #include "shared_decode.cuh"
 
@@ -142,6 +143,58 @@ moe_status launch_tc(const CUtensorMap& bmap, const TcArgs& a, cudaStream_t s) {
   return a.n_chunk > 64 ? launch_tc_epi<MODE, AF, 8>(bmap, a, s) : launch_tc_epi<MODE, AF, 4>(bmap, a, s);
 }
 
+// E2M1 plane of an MXFP4 weight array viewed by the block-scaled expert
+// kernel's loader: {columns (codes), rows, experts}, 128 x 128 boxes widened to
+// the f8f6f4 shared-memory layout (16U4_ALIGN16B), 128-byte swizzle.
+bool make_mx_weight_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr || base == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)a.cols, (cuuint64_t)a.rows, (cuuint64_t)a.E};
+  cuuint64_t strides[2] = {(cuuint64_t)a.cols / 2, (cuuint64_t)a.expert_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)kMxKT, 128, 1}, estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E4M3 token terms [rows][cols] bytes with a {128, 16} box, 128-byte swizzle.
+bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {(cuuint32_t)kMxKT, (cuuint32_t)kTcBoxRows}, estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One block-scaled expert launch (planned by mx_plan), one CTA per SM.
+template <int MODE, int G>
+moe_status launch_mx_g(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
+  static std::atomic<uint64_t> configured{0};
+  if (!smem_limit_once(configured, mx_expert_kernel<MODE, G>, kTcSmemMax)) return MOE_ERR_CUDA;
+  CUtensorMap w0, w1;
+  if (!make_mx_weight_map(&w0, a.w0, a)) return MOE_ERR_CUDA;
+  if (MODE == 0) {
+    if (!make_mx_weight_map(&w1, a.w1, a)) return MOE_ERR_CUDA;
+  } else {
+    w1 = w0;
+  }
+  mx_expert_kernel<MODE, G><<<sm_count(), kMxThreads, a.smem_bytes, s>>>(bmap, w0, w1, a);
+  return launch_status();
+}
+
+template <int MODE>
+moe_status launch_mx(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
+  switch (a.g) {
+    case 8: return launch_mx_g<MODE, 8>(bmap, a, s);
+    case 4: return launch_mx_g<MODE, 4>(bmap, a, s);
+    case 2: return launch_mx_g<MODE, 2>(bmap, a, s);
+    default: return launch_mx_g<MODE, 1>(bmap, a, s);
+  }
+}
+
 // Tokens per expert-kernel unit: the accumulator columns a unit reserves.  A
 // small chunk (few pairs per expert) leaves TMEM and shared memory for deeper
 // rings; a chunk below an expert's pair count makes its weights stream again.
@@ -149,6 +202,18 @@ int expert_chunk(int T, int K, int E) {
   const int64_t avg = ((int64_t)T * K + E - 1) / E;
   return avg <= 8 ? 32 : avg <= 24 ? 64 : kTcNMax;
 }
+
+// Path choice from the host-known T: with few pairs per expert (32-pair
+// chunks, decode) the weights stream through the block-scaled kernel; with
+// many, the kernel that dequantises to f16 keeps 128-token units, double the
+// epilogue warps and one read of each expert's weights.
+bool use_block_scaled(int T, int K, int E) { return expert_chunk(T, K, E) <= 32; }
+
+// E4M3 terms of the activations (exact for bf16) and of h between the GEMMs
+// on the block-scaled path: three terms of h for 32-pair chunks (N = 96).
+constexpr int kXTerms = 2;
+constexpr int kHTerms = 3;
+constexpr int kMxChunk = 32;
 
 // Router and shared expert run on the tensor cores above this token count
 // (and when their shapes fit the kernel's tiles).
@@ -344,28 +409,75 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  // x in pair order and f16 [T*top_k][hidden], then h in f16 [T*top_k][inter]
-  const size_t pairs = (size_t)T * dims->top_k;
-  return round_up(pairs * dims->hidden * 2, 256) + round_up(pairs * dims->inter * 2, 256);
+  const size_t pairs = (size_t)T * dims->top_k, H = dims->hidden, I = dims->inter;
+  // block-scaled path: E4M3 terms and E8M0 scales of the pairs' activations in
+  // expert order, then of h: [2][pairs][hidden], [2][pairs][hidden / 32],
+  // [3][pairs][inter], [3][pairs][inter / 32] bytes
+  const size_t mx = round_up(kXTerms * pairs * H, 256) + round_up(kXTerms * pairs * (H / 32), 256) +
+                    round_up(kHTerms * pairs * I, 256) + round_up(kHTerms * pairs * (I / 32), 256);
+  // dequantising path: the activations in expert order as f16 [pairs][hidden],
+  // then h in f16 [pairs][inter]
+  const size_t tc = round_up(pairs * H * 2, 256) + round_up(pairs * I * 2, 256);
+  return use_block_scaled(T, dims->top_k, dims->n_experts) ? mx : tc;
 }
 
-moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
-                           moe_mxfp4_proj up, moe_mxfp4_proj down, const int32_t* offsets,
-                           const int32_t* perm, float* y_perm, void* ws, size_t ws_bytes,
-                           void* stream) {
-  moe_status st = check_dims(dims);
-  if (st != MOE_OK) return st;
-  if (T < 0) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return MOE_OK;
-  if (!x || !offsets || !perm || !y_perm) return MOE_ERR_INVALID_ARG;
+namespace {
+
+moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t T, const moe_mxfp4_proj& gate,
+                                    const moe_mxfp4_proj& up, const moe_mxfp4_proj& down, const int32_t* offsets,
+                                    const int32_t* perm, float* y_perm, void* ws, cudaStream_t s) {
   const int H = dims->hidden, I = dims->inter;
-  if ((st = check_proj(gate, I, H)) != MOE_OK) return st;
-  if ((st = check_proj(up, I, H)) != MOE_OK) return st;
-  if ((st = check_proj(down, H, I)) != MOE_OK) return st;
-  if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
-  if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (I % 128 || H % 256 || H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
+  const int64_t pairs = (int64_t)T * dims->top_k;
+  uint8_t* xq = static_cast<uint8_t*>(ws);
+  uint8_t* xs = xq + round_up((size_t)kXTerms * pairs * H, 256);
+  uint8_t* hq = xs + round_up((size_t)kXTerms * pairs * (H / 32), 256);
+  uint8_t* hs = hq + round_up((size_t)kHTerms * pairs * I, 256);
+  MxArgs g{};
+  g.w0 = gate.base;
+  g.w1 = up.base;
+  g.expert_bytes = gate.expert_bytes;
+  g.rows = I;
+  g.cols = H;
+  g.offsets = offsets;
+  g.E = dims->n_experts;
+  g.pairs = (int)pairs;
+  g.parts = kXTerms;
+  g.b_scale = xs;
+  g.n_chunk = kMxChunk;
+  g.out = hq;
+  g.out_scale = hs;
+  g.out_parts = kHTerms;
+  g.limit = dims->swiglu_limit;
+  MxArgs d = g;
+  d.w0 = down.base;
+  d.w1 = nullptr;
+  d.expert_bytes = down.expert_bytes;
+  d.rows = H;
+  d.cols = I;
+  d.parts = kHTerms;
+  d.b_scale = hs;
+  d.out = y_perm;
+  d.out_scale = nullptr;
+  // shape check before anything is enqueued
+  if (!mx_plan(g, 0) || !mx_plan(d, 1) || gate.expert_bytes != up.expert_bytes) return MOE_ERR_UNSUPPORTED;
+  // the activations of every pair, in expert order, as E4M3 terms
+  const int64_t n8 = pairs * H / 8;
+  gather_split_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
+      static_cast<const uint4*>(x), perm, dims->top_k, H, pairs, kXTerms, xq, xs);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  CUtensorMap xmap, hmap;
+  if (!make_term_map(&xmap, xq, kXTerms * pairs, H) || !make_term_map(&hmap, hq, kHTerms * pairs, I))
+    return MOE_ERR_CUDA;
+  if ((st = launch_mx<0>(xmap, g, s)) != MOE_OK) return st;
+  return launch_mx<1>(hmap, d, s);
+}
+
+moe_status expert_gemm_dequant(const moe_dims* dims, const void* x, int32_t T, const moe_mxfp4_proj& gate,
+                               const moe_mxfp4_proj& up, const moe_mxfp4_proj& down, const int32_t* offsets,
+                               const int32_t* perm, float* y_perm, void* ws, cudaStream_t s) {
+  const int H = dims->hidden, I = dims->inter;
+  if (H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
   const int64_t pairs = (int64_t)T * dims->top_k;
   __half* x16 = static_cast<__half*>(ws);
   __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)pairs * H * 2, 256));
@@ -400,13 +512,38 @@ moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_m
   const int64_t n8 = pairs * H / 8;
   gather_f16_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
       static_cast<const uint4*>(x), perm, dims->top_k, H / 8, pairs, reinterpret_cast<uint4*>(x16));
-  if ((st = launch_status()) != MOE_OK) return st;
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
   if (!make_row_map(&xmap, x16, pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_row_map(&hmap, h16, pairs, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
   return launch_tc<1, kAMxfp4>(hmap, d, s);
+}
+
+}  // namespace
+
+moe_status moe_expert_gemm(const moe_dims* dims, const void* x, int32_t T, moe_mxfp4_proj gate,
+                           moe_mxfp4_proj up, moe_mxfp4_proj down, const int32_t* offsets,
+                           const int32_t* perm, float* y_perm, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !offsets || !perm || !y_perm) return MOE_ERR_INVALID_ARG;
+  const int H = dims->hidden, I = dims->inter;
+  if ((st = check_proj(gate, I, H)) != MOE_OK) return st;
+  if ((st = check_proj(up, I, H)) != MOE_OK) return st;
+  if ((st = check_proj(down, H, I)) != MOE_OK) return st;
+  if (!aligned(x, 16) || !aligned(y_perm, 16)) return MOE_ERR_ALIGNMENT;
+  if (ws == nullptr || ws_bytes < moe_expert_gemm_workspace_size(dims, T)) return MOE_ERR_WORKSPACE;
+  if (I % 128 || H % 256) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return use_block_scaled(T, dims->top_k, dims->n_experts)
+             ? expert_gemm_block_scaled(dims, x, T, gate, up, down, offsets, perm, y_perm, ws, s)
+             : expert_gemm_dequant(dims, x, T, gate, up, down, offsets, perm, y_perm, ws, s);
 }
 
 size_t shared_expert_workspace_size(const moe_dims* dims, int32_t T) {

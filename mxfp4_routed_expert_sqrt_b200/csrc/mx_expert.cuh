@@ -1,0 +1,565 @@
+// Grouped MXFP4 expert GEMM on the block-scaled tensor cores
+// (tcgen05.mma.kind::mxf8f6f4.block_scale), for every token count.
+//
+// The weights reach the MMA exactly as stored: E2M1 codes straight from HBM by
+// TMA (CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, which widens every 8 bytes of
+// packed codes to a 16-byte shared-memory chunk, the operand layout of the
+// f8f6f4 kind) and their E8M0 group-32 scales into tensor memory, where the MMA
+// applies them.  Nothing dequantises the weights in software.
+// ("ElytronAI / DeepSeek-v4-Flash", Layout and Sizes: the E2M1 nibble plane,
+// the E8M0 group-32 scale plane, expert xid at base + xid * expert_bytes;
+// "Model techniques map", row "SwiGLU feed-forward": the clamped SwiGLU.)
+//
+// The token operand is E4M3 with its own E8M0 group-32 scales.  Each
+// activation v is carried as a sum of `parts` E4M3 terms: term p encodes the
+// residual r_p = v - (terms 0 .. p-1) with the block scale 2^(floor(log2(max
+// |r_p| over the 32-value group)) - 7) and round-to-nearest-even.  Terms are
+// stacked along the MMA's N dimension (N = parts x tokens) and summed in fp32
+// by the epilogue.  Two terms carry a bf16 value exactly (8 significant bits
+// in two 4-bit terms) unless the residual of an element falls below the E4M3
+// normal range of its group; h between the GEMMs (fp32 in the epilogue) keeps
+// about 12 significant bits with three terms and about 8 with two.
+//
+// Per unit = (expert e, token chunk of <= n_chunk grouped pairs, row tile):
+//   MODE 0 (gate/up): acc0 = Wg[128 rows] x^T, acc1 = Wu[128 rows] x^T over
+//                     K = hidden; epilogue h = silu(min(g, L)) * clamp(u, -L, L)
+//                     written straight away as the down GEMM's E4M3 terms
+//   MODE 1 (down):    acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter; fp32 out
+// Swap-AB: weight rows are the MMA's M = 128, token terms its N.
+//
+// Pipeline stage = one K-tile of 128: both weight tiles (2 x 16 KB of shared
+// memory, 2 x 8 KB from HBM) and the unit's token rows of every term
+// (N x 128 bytes), all on one mbarrier; the MMA issuer runs 8 MMAs of K 32
+// and commits the stage back to the loader.  Scales travel in scale stages of
+// G K-tiles through tensor memory.
+//
+// Roles (320 threads, one CTA per SM, persistent over units):
+//   warps 0-3  epilogue (TMEM lane quadrant = warp): tcgen05.ld of the two
+//              accumulators, sum of the terms, SwiGLU and E4M3 split (MODE 0)
+//              or fp32 stores (MODE 1);
+//   warps 4-7  scale writers (lane quadrant = warp - 4): read the E8M0 bytes
+//              of the unit's weight rows and token terms with plain loads and
+//              tcgen05.st them in the layout the MMA reads (below), every
+//              quadrant holding a full copy;
+//   warp 8     loader (one thread): TMA boxes of weights and token terms;
+//   warp 9     TMEM owner and MMA issuer (one thread).
+// TMEM (512 columns): acc0 [0, acc), acc1 [acc, 2 acc), then the scale ring.
+// A scale stage holds, for K-tile j of the stage, the weight scales at column
+// 8j + 4m + c (m = tile, c = row / 32) and the token scales at column
+// 8G + 4j + c (c = N index / 32); lane i of every quadrant holds rows (or N
+// indices) 32c + i; byte b of a column is k-block 4 kt + b, which the MMA
+// selects with the scale-factor id.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp8.h>
+
+#include "tc_expert.cuh"
+
+namespace moe {
+
+constexpr int kMxThreads = 320;
+constexpr int kMxKT = 128;           // K of one pipeline stage (one TMA box of codes)
+constexpr int kMxTileBytes = 16384;  // shared-memory bytes of one 128 x 128 weight box
+constexpr int kMxTileTx = 8192;      // transaction bytes of that box (4 bits per code)
+constexpr int kMxMaxStages = 8;
+constexpr int kMxMaxSfStages = 4;
+constexpr int kMxMaxParts = 3;
+constexpr int kMxNMax = 128;   // MMA N: terms x padded tokens
+constexpr int kMxSfPerKt = 12; // TMEM columns per K-tile in a scale stage (8 weight + 4 token)
+
+struct MxArgs {
+  const uint8_t* w0;     // MODE 0: gate; MODE 1: down
+  const uint8_t* w1;     // MODE 0: up
+  int64_t expert_bytes;  // stride between experts
+  int rows;              // rows of one projection
+  int cols;              // columns (the reduction length K)
+  const int32_t* offsets;  // [E+1] grouped pairs
+  int E;
+  int pairs;             // token rows of one term
+  int parts;             // E4M3 terms of the token operand
+  const uint8_t* b_scale;  // token E8M0 [parts][pairs][cols / 32]
+  int n_chunk;           // tokens per unit: multiple of 16
+  void* out;             // MODE 0: E4M3 terms of h [out_parts][pairs][rows]; MODE 1: fp32 [pairs][rows]
+  uint8_t* out_scale;    // MODE 0: E8M0 of h [out_parts][pairs][rows / 32]
+  int out_parts;
+  float limit;
+  // filled in by mx_plan()
+  int g;             // K-tiles per scale stage
+  int acc_cols;      // TMEM columns per accumulator
+  int sf_stages;     // scale stages in TMEM
+  int stages;        // shared-memory stages
+  int stage_bytes;   // weights + token rows of one stage
+  int off_prefix;    // unit prefix + offsets copy
+  int smem_bytes;
+};
+
+// Ring depths and the shared-memory carve-up of one launch.  False when the
+// shape is outside what the kernel implements.
+inline bool mx_plan(MxArgs& a, int mode) {
+  const int nc = a.n_chunk;
+  if (nc < 16 || nc % 16 || a.parts < 1 || a.parts > kMxMaxParts || a.parts * nc > kMxNMax) return false;
+  if (mode == 0 && (a.out_parts < 1 || a.out_parts > kMxMaxParts)) return false;
+  if (a.cols % kMxKT || a.rows % (mode == 0 ? 128 : 256)) return false;
+  // 16U4_ALIGN16B tensor maps: strides in multiples of 32 bytes
+  if ((a.cols / 2) % 32 || a.expert_bytes % 32 || (a.cols / 32) % 4) return false;
+  const int nkt = a.cols / kMxKT;
+  a.g = nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt % 2 == 0 ? 2 : 1;
+  const int n = a.parts * nc;
+  a.acc_cols = (n + 31) / 32 * 32;
+  const int sf_cols = kMxSfPerKt * a.g;
+  a.sf_stages = (kTcTmemCols - 2 * a.acc_cols) / sf_cols;
+  if (a.sf_stages > kMxMaxSfStages) a.sf_stages = kMxMaxSfStages;
+  if (a.sf_stages < 1) return false;
+  a.stage_bytes = 2 * kMxTileBytes + n * 128;
+  const int pre = (2 * (a.E + 1) * 4 + 127) / 128 * 128;
+  const int budget = kTcSmemMax - 1024;
+  a.stages = (budget - pre) / a.stage_bytes;
+  if (a.stages > kMxMaxStages) a.stages = kMxMaxStages;
+  if (a.stages < 2) return false;
+  a.off_prefix = a.stages * a.stage_bytes;
+  a.smem_bytes = a.off_prefix + pre + 1024;
+  return a.smem_bytes <= kTcSmemMax;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both
+// K-major, E8M0 scales, fp32 D; scale-factor ids in bits 4-5 (B) and 29-30 (A).
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N) {
+  return (5u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= (A[smem] * SFA) (B[smem] * SFB)^T, scales from TMEM.
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+// G consecutive 32-bit words (4 * G bytes, 16-byte aligned for G >= 4).
+template <int G>
+__device__ __forceinline__ void load_words(const uint8_t* p, uint32_t* w) {
+  if constexpr (G == 8) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p)), b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else if constexpr (G == 4) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  } else if constexpr (G == 2) {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = a.x; w[1] = a.y;
+  } else {
+    w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+  }
+}
+
+// E8M0 block scale of a group whose largest magnitude has fp32 bits `amax`:
+// 2^(floor(log2 amax) - 7), so every |v| / scale is below 256 and rounds to at
+// most 256, inside the E4M3 range (448); 2^-127 for groups under 2^-120 (and
+// all-zero groups).
+__device__ __forceinline__ int e8m0_of_amax(uint32_t amax) { return max((int)(amax >> 23) - 7, 0); }
+// 2^(127 - s) and 2^(s - 127) for an E8M0 byte s in [0, 247]
+__device__ __forceinline__ float e8m0_inv(int s) { return __uint_as_float((uint32_t)(254 - s) << 23); }
+__device__ __forceinline__ float e8m0_val(int s) {
+  return s > 0 ? __uint_as_float((uint32_t)s << 23) : __uint_as_float(0x00400000u);
+}
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+  return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m3_val(uint32_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3)));
+}
+
+template <int MODE, int G>
+__global__ void __launch_bounds__(kMxThreads, 1)
+    mx_expert_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap0,
+                     const __grid_constant__ CUtensorMap wmap1, const MxArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kMxMaxStages], empty[kMxMaxStages];
+  __shared__ __align__(8) uint64_t sf_full[kMxMaxSfStages], sf_empty[kMxMaxSfStages];
+  __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
+  __shared__ uint32_t s_taddr;
+  __shared__ int32_t s_abort;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + args.off_prefix);  // [E + 1] units before group e
+  int32_t* s_off = s_prefix + args.E + 1;                                   // [E + 1] copy of offsets
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = args.E;
+  const int MT = MODE == 0 ? args.rows / 128 : args.rows / 256;  // row tiles per expert
+  const int nkt = args.cols / kMxKT;                             // K-tiles per unit
+  const int NC = args.n_chunk;
+  const int P = args.parts;
+  const int sr = args.cols / 32;  // E8M0 bytes per weight row and per token row
+  const uint32_t sf_base = 2 * args.acc_cols;
+  const int sf_cols = kMxSfPerKt * G;
+
+  // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
+  for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
+  __syncthreads();
+  if (warp == 0) {
+    int run = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int c = 0;
+      if (e < E) c = MT * ((s_off[e + 1] - s_off[e] + NC - 1) / NC);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < E) s_prefix[e] = run + incl - c;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_prefix[E] = run;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kMxMaxStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < kMxMaxSfStages; ++s) {
+      mbar_init(&sf_full[s], 4);  // one arrival per scale-writer warp
+      mbar_init(&sf_empty[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 4);
+    mbar_init(&mma_done, 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&s_taddr, kTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = s_taddr;
+  const int n_units = s_prefix[E];
+
+  // unit -> (expert, row tile, first grouped pair, tokens)
+  auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {  // last e with s_prefix[e] <= u
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    const int local = u - s_prefix[e];
+    mt = local % MT;
+    const int chunk = local / MT;
+    pos0 = s_off[e] + chunk * NC;
+    n = min(NC, s_off[e + 1] - pos0);
+  };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int32_t*>(&s_abort) != 0; };
+  auto give_up = [&]() {
+    set_error(kErrWaitTc);
+    *reinterpret_cast<volatile int32_t*>(&s_abort) = 1;
+  };
+  auto warp_wait = [&](uint64_t* bar, uint32_t ph) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, ph) ? 1 : 0) != 0;
+  };
+
+  if (warp == 8) {
+    // ------------------------------ loader -------------------------------------
+    if (lane == 0) {
+      TcRing rs(args.stages);
+      const uint64_t pol = policy_evict_first();
+      int issued = 0;
+      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        const int n16 = (n + 15) & ~15;  // rows past the chunk are loaded but never stored
+        const int y0 = MODE == 0 ? mt * 128 : mt * 256;
+        const int y1 = MODE == 0 ? mt * 128 : mt * 256 + 128;
+        const uint32_t tx = 2 * kMxTileTx + (uint32_t)(P * n16 * 128);
+        bool ok = true;
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[rs.s], tx);
+          uint8_t* dst = smem + rs.s * args.stage_bytes;
+          tma_load_3d(dst, &wmap0, kt * kMxKT, y0, e, &full[rs.s], pol);
+          tma_load_3d(dst + kMxTileBytes, MODE == 0 ? &wmap1 : &wmap0, kt * kMxKT, y1, e, &full[rs.s], pol);
+          uint8_t* bdst = dst + 2 * kMxTileBytes;
+          for (int p = 0; p < P; ++p)
+            for (int j = 0; j < n16; j += kTcBoxRows)
+              tma_load_2d(bdst + (p * n16 + j) * 128, &bmap, kt * kMxKT, p * args.pairs + pos0 + j, &full[rs.s]);
+          rs.next();
+          ++issued;
+        }
+        if (!ok) break;
+      }
+      // the last fills must have landed before the CTA exits
+      for (int i = 0; i < min(issued, rs.n); ++i) {
+        const int s = (rs.s - 1 - i + rs.n) % rs.n;
+        if (!mbar_wait(&full[s], s < rs.s ? rs.ph : rs.ph ^ 1)) set_error(kErrWaitTc);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------ MMA issuer ----------------------------------
+    if (lane == 0) {
+      TcRing rs(args.stages), rf(args.sf_stages);
+      uint32_t un = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok && !aborted(); u += gridDim.x, ++un) {
+        int e, mt, pos0, n;
+        decode_unit(u, e, mt, pos0, n);
+        const int n16 = (n + 15) & ~15;
+        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, P * n16);
+        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int j = kt % G;
+          if (j == 0 && !mbar_wait(&sf_full[rf.s], rf.ph)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&full[rs.s], rs.ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t wa = smem_u32(smem + rs.s * args.stage_bytes), ba = wa + 2 * kMxTileBytes;
+          const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
+            const uint32_t sel = (uint32_t)kb << 30;
+            const uint64_t bd = sdesc_sw128(ba + kb * 32);
+            const uint32_t sfb = (sfc + 8 * G + 4 * j) | sel;
+            const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+            umma_mx(tbase, sdesc_sw128(wa + kb * 32), bd, id, acc, (sfc + 8 * j) | sel, sfb);
+            umma_mx(tbase + args.acc_cols, sdesc_sw128(wa + kMxTileBytes + kb * 32), bd, id, acc,
+                    (sfc + 8 * j + 4) | sel, sfb);
+          }
+          umma_commit(&empty[rs.s]);
+          rs.next();
+          if (j == G - 1) {
+            umma_commit(&sf_empty[rf.s]);
+            rf.next();
+          }
+          if (kt == nkt - 1) umma_commit(&acc_full);
+        }
+      }
+      if (!ok) give_up();
+      // every MMA of this thread done before TMEM is released
+      umma_commit(&mma_done);
+      if (!mbar_wait(&mma_done, 0)) set_error(kErrWaitTc);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------ scale writers --------------------------------
+    const int q = warp & 3;
+    const uint32_t lrow = (uint32_t)(q * 32) << 16;
+    const int64_t plane = (int64_t)args.rows * (args.cols / 2);
+    TcRing rf(args.sf_stages);
+    for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      bool ok = true;
+      for (int g = 0; g < nkt / G; ++g) {
+        // weight scales: a[8 j + 4 m + c] = bytes 4 (G g + j) .. +3 of row 32 c + lane of tile m
+        uint32_t a[8 * G], b[4 * G];
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int R = MODE == 0 ? mt * 128 + 32 * c + lane : mt * 256 + 128 * m + 32 * c + lane;
+            const uint8_t* src = (MODE == 0 && m == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes + plane +
+                                 (int64_t)R * sr + 4 * G * g;
+            uint32_t w[G];
+            load_words<G>(src, w);
+#pragma unroll
+            for (int j = 0; j < G; ++j) a[8 * j + 4 * m + c] = w[j];
+          }
+        // token scales: b[4 j + c] for N index 32 c + lane = term p, token t
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int nn = 32 * c + lane, p = nn / n16, t = nn - p * n16;
+          uint32_t w[G];
+#pragma unroll
+          for (int j = 0; j < G; ++j) w[j] = 0;
+          if (p < P && t < n)
+            load_words<G>(args.b_scale + ((int64_t)p * args.pairs + pos0 + t) * sr + 4 * G * g, w);
+#pragma unroll
+          for (int j = 0; j < G; ++j) b[4 * j + c] = w[j];
+        }
+        if (!warp_wait(&sf_empty[rf.s], rf.ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t col = tbase + lrow + sf_base + rf.s * sf_cols;
+#pragma unroll
+        for (int i = 0; i < G; ++i) tmem_st8(col + 8 * i, a + 8 * i);
+        if constexpr (G == 1) {  // 4 token-scale columns
+          asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(col + 8), "r"(b[0]),
+                       "r"(b[1]), "r"(b[2]), "r"(b[3])
+                       : "memory");
+        } else {
+#pragma unroll
+          for (int i = 0; i < G / 2; ++i) tmem_st8(col + 8 * G + 8 * i, b + 8 * i);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[rf.s]);
+        rf.next();
+      }
+      if (!ok) {
+        give_up();
+        break;
+      }
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------------
+    const int q = warp;  // TMEM lanes 32q .. 32q + 31
+    const uint32_t lrow = (uint32_t)(q * 32) << 16;
+    uint32_t un = 0;
+    for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x, ++un) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      if (!warp_wait(&acc_full, un & 1)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      for (int c0 = 0; c0 < n; c0 += 16) {
+        float g[16], v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) g[j] = v[j] = 0.f;
+        for (int p = 0; p < P; ++p) {  // sum of the token terms
+          uint32_t t0[16], t1[16];
+          tmem_ld16(tbase + lrow + p * n16 + c0, t0);
+          tmem_ld16(tbase + lrow + args.acc_cols + p * n16 + c0, t1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            g[j] += __uint_as_float(t0[j]);
+            v[j] += __uint_as_float(t1[j]);
+          }
+        }
+        if (MODE == 0) {
+          // h of row col for 16 tokens, split into E4M3 terms; the 32 lanes of
+          // the warp are one group of 32 h values of a token (the down GEMM's k)
+          const int col = mt * 128 + q * 32 + lane;
+          uint8_t* hq = static_cast<uint8_t*>(args.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n) {  // the same for the whole warp
+              float r = silu_clamped_swiglu(g[j], v[j], args.limit);
+              const int64_t pos = pos0 + c0 + j;
+              for (int p = 0; p < args.out_parts; ++p) {
+                const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r)));
+                const int s = e8m0_of_amax(amax);
+                const uint32_t code = e4m3_rn(r * e8m0_inv(s));
+                const int64_t row = (int64_t)p * args.pairs + pos;
+                hq[row * args.rows + col] = (uint8_t)code;
+                if (lane == 0) args.out_scale[row * (args.rows / 32) + col / 32] = (uint8_t)s;
+                r -= e4m3_val(code) * e8m0_val(s);
+              }
+            }
+        } else {
+          float* out = static_cast<float*>(args.out);
+          const int col = mt * 256 + q * 32 + lane;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n) {
+              out[(int64_t)(pos0 + c0 + j) * args.rows + col] = g[j];
+              out[(int64_t)(pos0 + c0 + j) * args.rows + col + 128] = v[j];
+            }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTcTmemCols);
+  }
+}
+
+// Activations of every pair in expert order as `parts` E4M3 terms with E8M0
+// group-32 scales: q[p][pos][k], sc[p][pos][k / 32] for x[perm[pos] / top_k].
+// One thread per 8 values; the 4 threads of a 32-value group are adjacent lanes.
+__global__ void gather_split_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int top_k,
+                                    int hidden, int64_t pairs, int parts, uint8_t* __restrict__ q,
+                                    uint8_t* __restrict__ sc) {
+  const int h8 = hidden / 8;
+  const int64_t n = pairs * h8;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n; base += stride) {
+    const int64_t i = base + lane;
+    const bool ok = i < n;  // whole 4-lane groups: n is a multiple of 4
+    float v[8];
+    int64_t pos = 0;
+    int c8 = 0;
+    if (ok) {
+      pos = i / h8;
+      c8 = (int)(i - pos * h8);
+      const int64_t t = perm[pos] / top_k;
+      const uint4 w = x[t * h8 + c8];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(ws[k] << 16);
+        v[2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = 0.f;
+    }
+    for (int p = 0; p < parts; ++p) {
+      uint32_t amax = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) amax = max(amax, __float_as_uint(fabsf(v[k])));
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const int s = e8m0_of_amax(amax);
+      const float inv = e8m0_inv(s), val = e8m0_val(s);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t code = e4m3_rn(v[k] * inv);
+        if (k < 4) lo |= code << (8 * k);
+        else hi |= code << (8 * (k - 4));
+        v[k] -= e4m3_val(code) * val;
+      }
+      if (ok) {
+        const int64_t row = (int64_t)p * pairs + pos;
+        reinterpret_cast<uint2*>(q + row * hidden)[c8] = make_uint2(lo, hi);
+        if ((c8 & 3) == 0) sc[row * (hidden / 32) + c8 / 4] = (uint8_t)s;
+      }
+    }
+  }
+}
+
+}  // namespace moe

@@ -178,10 +178,12 @@ def _expert_gemm(dc, T):
     return idx, perm.cpu().numpy()[:T * K], y[:T * K * H].view(T * K, H).cpu().numpy()
 
 
-# The call picks its token chunk (32, 64 or 128 pairs per unit) from the mean
-# pairs per expert; the zipf case piles most pairs onto a few experts, so their
-# groups span many 32-pair chunks, and it samples both sides of every chunk
-# boundary of the most loaded expert.
+# The call picks its path and token chunk from the mean pairs per expert: at
+# most 8 runs the block-scaled kernel in 32-pair chunks (every case here up to
+# v4_T300 and the tiny T8/T37 ones), more runs the dequantising kernel in 64-
+# or 128-pair chunks (tiny T100/T1000).  The zipf case piles most pairs onto a
+# few experts, so their groups span many 32-pair chunks, and it samples both
+# sides of every chunk boundary of the most loaded expert.
 EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64, None), ("tiny_T37", gen.TINY, 37, 74, None),
                 ("v4_T1", gen.V4, 1, 6, None), ("v4_T8", gen.V4, 8, 48, None), ("v4_T37", gen.V4, 37, 24, None),
                 ("v4_T64", gen.V4, 64, 24, None), ("tiny_T100_tc", gen.TINY, 100, 200, None),

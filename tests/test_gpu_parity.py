@@ -188,7 +188,11 @@ EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64, None), ("tiny_T37", gen.TINY, 37, 7
                 ("v4_T1", gen.V4, 1, 6, None), ("v4_T8", gen.V4, 8, 48, None), ("v4_T37", gen.V4, 37, 24, None),
                 ("v4_T64", gen.V4, 64, 24, None), ("tiny_T100_tc", gen.TINY, 100, 200, None),
                 ("tiny_T1000_tc", gen.TINY, 1000, 120, None), ("v4_T96_tc", gen.V4, 96, 24, None),
-                ("v4_T300_tc", gen.V4, 300, 24, None), ("v4_zipf_T256_chunks", gen.V4, 256, 16, "zipf")]
+                ("v4_T300_tc", gen.V4, 300, 24, None), ("v4_zipf_T256_chunks", gen.V4, 256, 16, "zipf"),
+                # the two sides of the path switch: 8 pairs per expert on average
+                # (the largest block-scaled call), then 9 (the smallest dequantising one)
+                ("v4_T341_block_scaled_max", gen.V4, 341, 24, None),
+                ("v4_T342_dequant_min", gen.V4, 342, 24, None)]
 
 
 @pytest.mark.parametrize("name,dims,T,nsample,bias", EXPERT_CASES, ids=[c[0] for c in EXPERT_CASES])

@@ -169,12 +169,22 @@ def oracle_sample(dims, seed, layer, x_bits, router, bias, shared, tok=None, tab
 
 
 def time_oracle(dims, x_bits, router, bias, blobs, shared, tok=None, table=None):
+    """Seconds of one fp64 oracle pass over x_bits, the threads it used, its output."""
     import oracle
     nthreads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    oracle.moe_layer(dims, x_bits, np.arange(x_bits.shape[0]), router, bias, *blobs, shared=shared, tok=tok,
-                     table=table, nthreads=nthreads)
-    return time.perf_counter() - t0, nthreads
+    out, _, _ = oracle.moe_layer(dims, x_bits, np.arange(x_bits.shape[0]), router, bias, *blobs, shared=shared,
+                                 tok=tok, table=table, nthreads=nthreads)
+    return time.perf_counter() - t0, nthreads, out
+
+
+def parity_stats(got, want):
+    """The layer tolerance's two figures for a sample: max|err| / RMS(want) and
+    sum|err| / sum|want|."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want)
+    return float(err.max() / np.sqrt(np.mean(want ** 2))), float(err.sum() / np.abs(want).sum())
 
 
 def sample_inputs(dims, spec_batches, seed, n_tok):
@@ -202,7 +212,7 @@ def run_reference(args, dims, batches, desc, metric, unit):
     total, threads = 0.0, 1
     for i in range(args.warmup + args.steps):
         s = i % 4
-        dt, threads = time_oracle(dims, xs[s], router, None, blobs[s], shared, toks[s], table)
+        dt, threads, _ = time_oracle(dims, xs[s], router, None, blobs[s], shared, toks[s], table)
         if i >= args.warmup:
             total += dt
     value = n_per_step * args.steps / total
@@ -219,6 +229,11 @@ def run_reference(args, dims, batches, desc, metric, unit):
 # ---------------------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------------------
+
+# B200 specification peaks, reported beside the measured ones: HBM3e ~8 TB/s,
+# dense bf16 2.25 PFLOP/s
+SPEC_HBM_GBS = 8000.0
+SPEC_BF16_TFLOPS = 2250.0
 
 # moe_expert_gemm runs the block-scaled kernel when an expert averages at most
 # 8 pairs (the library's path choice from T), else the dequantising kernel.
@@ -450,6 +465,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         achieved = flops / (k_ms / 1e3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                    "spec_peak": SPEC_BF16_TFLOPS, "frac_spec": round(achieved / SPEC_BF16_TFLOPS, 4),
                     "kernel": kernel, "algorithmic_flops_per_launch": int(flops / n_calls),
                     "avg_launch_ms": round(k_ms / n_calls, 5)}
     else:
@@ -459,6 +475,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         achieved = k_bytes / (k_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                    "spec_peak": SPEC_HBM_GBS, "frac_spec": round(achieved / SPEC_HBM_GBS, 4),
                     "kernel": kernel, "algorithmic_bytes_per_launch": int(k_bytes / n_calls),
                     "avg_launch_ms": round(k_ms / n_calls, 5)}
 
@@ -496,6 +513,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     assert m.moe_device_error() == 0
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_tok = 8 if args.workload != "tiny" else 8
         B, l = batches[-1]
@@ -505,9 +523,30 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         if hashed:
             tok = toksets[(len(batches) - 1, 0)].cpu().numpy()[:n_tok]
         blobs = oracle_sample(dims, seed, l, xs, lay.router_np, lay.bias_np, lay.shared_np, tok, lay.table_np)
-        dt, threads = time_oracle(dims, xs, lay.router_np, lay.bias_np, blobs, lay.shared_np, tok, lay.table_np)
+        dt, threads, want = time_oracle(dims, xs, lay.router_np, lay.bias_np, blobs, lay.shared_np, tok,
+                                        lay.table_np)
         cpu = {"value": n_tok / dt, "unit": unit, "cores": threads, "kind": "oracle",
                "sample": f"{n_tok} tokens of the batch-{B} layer (x set 0), whole layer in fp64"}
+        # the same sample through the CUDA layer (untimed), against the oracle's
+        # output; a failure here is reported in the line, not fatal to it
+        try:
+            jl = len(batches) - 1
+            out_s = torch.empty(n_tok * H, dtype=torch.float32, device=dev)
+            runners[jl].forward(lay.w, xsets[(jl, 0)][1][:n_tok], n_tok, out_s,
+                                token_ids=toksets[(jl, 0)][:n_tok] if hashed else None)
+            torch.cuda.synchronize()
+            dev_err = m.moe_device_error()
+            mx_err, l1_err = parity_stats(out_s.view(n_tok, H).cpu().numpy(), want)
+            parity = {"sample": cpu["sample"], "max_err_over_rms": mx_err, "sum_err_over_sum_ref": l1_err,
+                      "tolerance": {"max_err_over_rms": 1e-2, "sum_err_over_sum_ref": 2e-3},
+                      "device_error": dev_err}
+            if not hashed:  # the bench's x sets are not redrawn: how close routing came to a tie
+                import oracle
+                _, _, _, gap = oracle.route(xs, lay.router_np, lay.bias_np, K, dims.route_scale)
+                parity["min_topk_gap"] = float(gap.min())
+                parity["tokens_with_gap_below_1e-4"] = int((gap <= 1e-4).sum())
+        except Exception as exc:  # noqa: BLE001
+            parity = {"error": repr(exc)[:300]}
 
     clocks = sampler.summary(wall0, wall1)
     for g, _, _, _ in timed:
@@ -524,7 +563,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
                            "l2": "inputs larger than L2: each step streams distinct expert weights "
                                  "of resident layers (no flush)",
                            "cuda_graphs": True, "zipf_kappa": kappa},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
                 "gpu_launches": n_layer_kernels * len(batches) * args.steps,
                 "clocks": clocks}
         print(json.dumps(line), flush=True)

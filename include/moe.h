@@ -188,7 +188,9 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *  offsets, perm  as written by moe_permute.
  *  y_perm   fp32 [T*top_k][hidden] out.
  *  ws       device workspace of moe_expert_gemm_workspace_size(dims, T)
- *           bytes (its layout depends on the path below).
+ *           bytes: the block-scaled path's layout below, of which the
+ *           dequantising path uses a prefix, so the size grows with T and a
+ *           workspace sized for some T serves every smaller T.
  * Two paths, chosen from T alone (mean pairs per expert, ceil(T*top_k / E)):
  *  - at most 8 (decode): block-scaled tensor-core MMAs
  *    (tcgen05 kind::mxf8f6f4): the E2M1 codes and E8M0 scales go to the

@@ -410,15 +410,15 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
   const size_t pairs = (size_t)T * dims->top_k, H = dims->hidden, I = dims->inter;
-  // block-scaled path: E4M3 terms and E8M0 scales of the pairs' activations in
-  // expert order, then of h: [2][pairs][hidden], [2][pairs][hidden / 32],
-  // [3][pairs][inter], [3][pairs][inter / 32] bytes
-  const size_t mx = round_up(kXTerms * pairs * H, 256) + round_up(kXTerms * pairs * (H / 32), 256) +
-                    round_up(kHTerms * pairs * I, 256) + round_up(kHTerms * pairs * (I / 32), 256);
-  // dequantising path: the activations in expert order as f16 [pairs][hidden],
-  // then h in f16 [pairs][inter]
-  const size_t tc = round_up(pairs * H * 2, 256) + round_up(pairs * I * 2, 256);
-  return use_block_scaled(T, dims->top_k, dims->n_experts) ? mx : tc;
+  // The block-scaled path's layout: E4M3 terms and E8M0 scales of the pairs'
+  // activations in expert order, then of h: [2][pairs][hidden],
+  // [2][pairs][hidden / 32], [3][pairs][inter], [3][pairs][inter / 32] bytes.
+  // The dequantising path uses a prefix of it (x in f16 [pairs][hidden], then
+  // h in f16 [pairs][inter]: hidden / 16 + inter + 3 inter / 32 bytes fewer
+  // per pair), so the size grows with T whichever path T selects and a
+  // workspace sized for some T serves every smaller T.
+  return round_up(kXTerms * pairs * H, 256) + round_up(kXTerms * pairs * (H / 32), 256) +
+         round_up(kHTerms * pairs * I, 256) + round_up(kHTerms * pairs * (I / 32), 256);
 }
 
 namespace {

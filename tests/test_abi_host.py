@@ -66,17 +66,22 @@ def _r256(n):
 
 @pytest.mark.parametrize("dims,T", [(gen.V4, 1), (gen.V4, 64), (gen.V4, 341), (gen.V4, 342), (gen.V4, 4096),
                                     (gen.TINY, 8), (gen.TINY, 64), (gen.TINY, 65), (gen.TINY, 1000)])
-def test_expert_gemm_workspace_follows_the_path_choice(m, dims, T):
-    """At most 8 pairs per expert on average (ceil(T*K/E)) runs the block-scaled
-    path: E4M3 terms and E8M0 scales of x (2 terms) and of h (3 terms); above,
-    the dequantising path: x and h in f16 (the layouts moe.h documents)."""
+def test_expert_gemm_workspace_covers_both_paths(m, dims, T):
+    """The block-scaled path's layout (E4M3 terms and E8M0 scales of x, 2 terms,
+    and of h, 3 terms) for every T: it is larger than the dequantising path's
+    (x and h in f16), so the size grows with T across the switch from one path
+    to the other (moe.h)."""
     H, I, E, K = dims.hidden, dims.inter, dims.n_experts, dims.top_k
     P = T * K
-    if -(-P // E) <= 8:
-        want = _r256(2 * P * H) + _r256(2 * P * (H // 32)) + _r256(3 * P * I) + _r256(3 * P * (I // 32))
-    else:
-        want = _r256(P * H * 2) + _r256(P * I * 2)
+    want = _r256(2 * P * H) + _r256(2 * P * (H // 32)) + _r256(3 * P * I) + _r256(3 * P * (I // 32))
+    assert want >= _r256(P * H * 2) + _r256(P * I * 2)
     assert m.moe_expert_gemm_workspace_size(dims, T) == want
+
+
+def test_expert_gemm_workspace_grows_with_T(m):
+    for dims in (gen.V4, gen.TINY):
+        sizes = [m.moe_expert_gemm_workspace_size(dims, T) for T in range(0, 700)]
+        assert all(a <= b for a, b in zip(sizes, sizes[1:]))
 
 
 def test_argument_errors_return_before_launch(m):

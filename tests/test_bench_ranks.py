@@ -65,3 +65,14 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(None, 3.5, "cpu") == 3.5
     assert bench.whole_job_rate(1, 105, 50, 0.1) == pytest.approx(52500.0)
+
+
+def test_parity_stats_are_the_tolerance_figures():
+    import numpy as np
+    import bench
+    want = np.array([[3.0, -4.0], [0.0, 5.0]])  # RMS = sqrt(50 / 4)
+    got = want + np.array([[0.5, 0.0], [0.0, -0.25]])
+    mx, l1 = bench.parity_stats(got, want)
+    assert np.isclose(mx, 0.5 / np.sqrt(12.5))
+    assert np.isclose(l1, 0.75 / 12.0)
+    assert bench.parity_stats(want, want) == (0.0, 0.0)

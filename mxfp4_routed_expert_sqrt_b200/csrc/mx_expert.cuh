@@ -120,7 +120,9 @@ inline bool mx_plan(MxArgs& a, int mode) {
   if (a.stages < 2) return false;
   a.off_prefix = a.stages * a.stage_bytes;
   a.smem_bytes = a.off_prefix + pre + 1024;
-  return a.smem_bytes <= kTcSmemMax;
+  // every CTA allocates all 512 TMEM columns, so no second CTA may share its
+  // SM: more than half of the SM's shared memory guarantees that
+  return a.smem_bytes <= kTcSmemMax && a.smem_bytes > kTcSmemMax / 2;
 }
 
 // Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both

@@ -1,0 +1,143 @@
+// Launch arguments of moe_expert_gemm's two paths, on the host only (no CUDA
+// call): the path choice from T, the token chunk, the E4M3 term counts, the
+// workspace carve-up and the pipeline plans.  moe_expert_gemm launches what
+// these functions fill in; a CPU test checks them for every token count.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "mx_expert.cuh"
+#include "tc_expert.cuh"
+
+namespace moe {
+
+inline size_t ws_round_up(size_t v) { return (v + 255) / 256 * 256; }
+
+// Tokens per expert-kernel unit: the accumulator columns a unit reserves.  A
+// small chunk (few pairs per expert) leaves TMEM and shared memory for deeper
+// rings; a chunk below an expert's pair count makes its weights stream again.
+inline int expert_chunk(int T, int K, int E) {
+  const int64_t avg = ((int64_t)T * K + E - 1) / E;
+  return avg <= 8 ? 32 : avg <= 24 ? 64 : kTcNMax;
+}
+
+// Path choice from the host-known T: with few pairs per expert (32-pair
+// chunks, decode) the weights stream through the block-scaled kernel; with
+// many, the kernel that dequantises to f16 keeps 128-token units, double the
+// epilogue warps and one read of each expert's weights.
+inline bool use_block_scaled(int T, int K, int E) { return expert_chunk(T, K, E) <= 32; }
+
+// E4M3 terms of the activations (exact for bf16) and of h between the GEMMs
+// on the block-scaled path: three terms of h for 32-pair chunks (N = 96).
+constexpr int kXTerms = 2;
+constexpr int kHTerms = 3;
+constexpr int kMxChunk = 32;
+
+// The block-scaled path's workspace: E4M3 terms and E8M0 scales of the pairs'
+// activations in expert order, then of h: [2][pairs][hidden],
+// [2][pairs][hidden / 32], [3][pairs][inter], [3][pairs][inter / 32] bytes.
+// The dequantising path uses a prefix of it (x in f16 [pairs][hidden], then
+// h in f16 [pairs][inter]: hidden / 16 + inter + 3 inter / 32 bytes fewer per
+// pair), so the size grows with T whichever path T selects and a workspace
+// sized for some T serves every smaller T.
+inline size_t expert_gemm_ws_bytes(const moe_dims& dims, int T) {
+  const size_t pairs = (size_t)T * dims.top_k, H = dims.hidden, I = dims.inter;
+  return ws_round_up(kXTerms * pairs * H) + ws_round_up(kXTerms * pairs * (H / 32)) +
+         ws_round_up(kHTerms * pairs * I) + ws_round_up(kHTerms * pairs * (I / 32));
+}
+
+// Block-scaled path: both launches' arguments (planned) and the workspace
+// buffers they use.
+struct MxLaunch {
+  MxArgs g, d;                   // gate/up + SwiGLU, down
+  uint8_t *xq, *xs, *hq, *hs;    // E4M3 terms and E8M0 scales of x and of h
+  int64_t pairs;
+};
+
+// False when the shape is outside the kernel (nothing may be launched then).
+inline bool mx_launch_args(const moe_dims& dims, int T, const moe_mxfp4_proj& gate, const moe_mxfp4_proj& up,
+                           const moe_mxfp4_proj& down, const int32_t* offsets, float* y_perm, void* ws,
+                           MxLaunch& L) {
+  const int H = dims.hidden, I = dims.inter;
+  L.pairs = (int64_t)T * dims.top_k;
+  L.xq = static_cast<uint8_t*>(ws);
+  L.xs = L.xq + ws_round_up((size_t)kXTerms * L.pairs * H);
+  L.hq = L.xs + ws_round_up((size_t)kXTerms * L.pairs * (H / 32));
+  L.hs = L.hq + ws_round_up((size_t)kHTerms * L.pairs * I);
+  MxArgs& g = L.g;
+  g = MxArgs{};
+  g.w0 = gate.base;
+  g.w1 = up.base;
+  g.expert_bytes = gate.expert_bytes;
+  g.rows = I;
+  g.cols = H;
+  g.offsets = offsets;
+  g.E = dims.n_experts;
+  g.pairs = (int)L.pairs;
+  g.parts = kXTerms;
+  g.b_scale = L.xs;
+  g.n_chunk = kMxChunk;
+  g.out = L.hq;
+  g.out_scale = L.hs;
+  g.out_parts = kHTerms;
+  g.limit = dims.swiglu_limit;
+  MxArgs& d = L.d;
+  d = g;
+  d.w0 = down.base;
+  d.w1 = nullptr;
+  d.expert_bytes = down.expert_bytes;
+  d.rows = H;
+  d.cols = I;
+  d.parts = kHTerms;
+  d.b_scale = L.hs;
+  d.out = y_perm;
+  d.out_scale = nullptr;
+  return mx_plan(g, 0) && mx_plan(d, 1) && gate.expert_bytes == up.expert_bytes;
+}
+
+// Dequantising path: both launches' arguments (each launch plans its own
+// copy) and the f16 buffers of x and h.
+struct TcLaunch {
+  TcArgs g, d;
+  __half *x16, *h16;
+  int64_t pairs;
+};
+
+inline bool tc_launch_args(const moe_dims& dims, int T, const moe_mxfp4_proj& gate, const moe_mxfp4_proj& up,
+                           const moe_mxfp4_proj& down, const int32_t* offsets, float* y_perm, void* ws,
+                           TcLaunch& L) {
+  const int H = dims.hidden, I = dims.inter;
+  if (H % 64 || I % 64) return false;
+  L.pairs = (int64_t)T * dims.top_k;
+  L.x16 = static_cast<__half*>(ws);
+  L.h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + ws_round_up((size_t)L.pairs * H * 2));
+  TcArgs& g = L.g;
+  g = TcArgs{};
+  g.w0 = gate.base;
+  g.w1 = up.base;
+  g.expert_bytes = gate.expert_bytes;
+  g.rows = I;
+  g.a_cols = H;
+  g.k_total = H;
+  g.b_cols = H;
+  g.offsets = offsets;
+  g.E = dims.n_experts;
+  g.n_chunk = expert_chunk(T, dims.top_k, dims.n_experts);
+  g.out = L.h16;
+  g.limit = dims.swiglu_limit;
+  TcArgs& d = L.d;
+  d = g;
+  d.w0 = down.base;
+  d.w1 = nullptr;
+  d.expert_bytes = down.expert_bytes;
+  d.rows = H;
+  d.a_cols = I;
+  d.k_total = I;
+  d.b_cols = I;
+  d.out = y_perm;
+  TcArgs pg = g, pd = d;  // the shape check; the launches plan their own copies
+  return tc_plan(pg, kAMxfp4) && tc_plan(pd, kAMxfp4);
+}
+
+}  // namespace moe

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "expert_launch.h"
 #include "mx_expert.cuh"
 #include "tc_expert.cuh"
 #include "shared_decode.cuh"
@@ -194,26 +195,6 @@ moe_status launch_mx(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
     default: return launch_mx_g<MODE, 1>(bmap, a, s);
   }
 }
-
-// Tokens per expert-kernel unit: the accumulator columns a unit reserves.  A
-// small chunk (few pairs per expert) leaves TMEM and shared memory for deeper
-// rings; a chunk below an expert's pair count makes its weights stream again.
-int expert_chunk(int T, int K, int E) {
-  const int64_t avg = ((int64_t)T * K + E - 1) / E;
-  return avg <= 8 ? 32 : avg <= 24 ? 64 : kTcNMax;
-}
-
-// Path choice from the host-known T: with few pairs per expert (32-pair
-// chunks, decode) the weights stream through the block-scaled kernel; with
-// many, the kernel that dequantises to f16 keeps 128-token units, double the
-// epilogue warps and one read of each expert's weights.
-bool use_block_scaled(int T, int K, int E) { return expert_chunk(T, K, E) <= 32; }
-
-// E4M3 terms of the activations (exact for bf16) and of h between the GEMMs
-// on the block-scaled path: three terms of h for 32-pair chunks (N = 96).
-constexpr int kXTerms = 2;
-constexpr int kHTerms = 3;
-constexpr int kMxChunk = 32;
 
 // Router and shared expert run on the tensor cores above this token count
 // (and when their shapes fit the kernel's tiles).
@@ -409,16 +390,7 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   if (dims == nullptr || T < 0) return 0;
-  const size_t pairs = (size_t)T * dims->top_k, H = dims->hidden, I = dims->inter;
-  // The block-scaled path's layout: E4M3 terms and E8M0 scales of the pairs'
-  // activations in expert order, then of h: [2][pairs][hidden],
-  // [2][pairs][hidden / 32], [3][pairs][inter], [3][pairs][inter / 32] bytes.
-  // The dequantising path uses a prefix of it (x in f16 [pairs][hidden], then
-  // h in f16 [pairs][inter]: hidden / 16 + inter + 3 inter / 32 bytes fewer
-  // per pair), so the size grows with T whichever path T selects and a
-  // workspace sized for some T serves every smaller T.
-  return round_up(kXTerms * pairs * H, 256) + round_up(kXTerms * pairs * (H / 32), 256) +
-         round_up(kHTerms * pairs * I, 256) + round_up(kHTerms * pairs * (I / 32), 256);
+  return expert_gemm_ws_bytes(*dims, T);
 }
 
 namespace {
@@ -426,100 +398,43 @@ namespace {
 moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t T, const moe_mxfp4_proj& gate,
                                     const moe_mxfp4_proj& up, const moe_mxfp4_proj& down, const int32_t* offsets,
                                     const int32_t* perm, float* y_perm, void* ws, cudaStream_t s) {
-  const int H = dims->hidden, I = dims->inter;
-  const int64_t pairs = (int64_t)T * dims->top_k;
-  uint8_t* xq = static_cast<uint8_t*>(ws);
-  uint8_t* xs = xq + round_up((size_t)kXTerms * pairs * H, 256);
-  uint8_t* hq = xs + round_up((size_t)kXTerms * pairs * (H / 32), 256);
-  uint8_t* hs = hq + round_up((size_t)kHTerms * pairs * I, 256);
-  MxArgs g{};
-  g.w0 = gate.base;
-  g.w1 = up.base;
-  g.expert_bytes = gate.expert_bytes;
-  g.rows = I;
-  g.cols = H;
-  g.offsets = offsets;
-  g.E = dims->n_experts;
-  g.pairs = (int)pairs;
-  g.parts = kXTerms;
-  g.b_scale = xs;
-  g.n_chunk = kMxChunk;
-  g.out = hq;
-  g.out_scale = hs;
-  g.out_parts = kHTerms;
-  g.limit = dims->swiglu_limit;
-  MxArgs d = g;
-  d.w0 = down.base;
-  d.w1 = nullptr;
-  d.expert_bytes = down.expert_bytes;
-  d.rows = H;
-  d.cols = I;
-  d.parts = kHTerms;
-  d.b_scale = hs;
-  d.out = y_perm;
-  d.out_scale = nullptr;
+  MxLaunch L;
   // shape check before anything is enqueued
-  if (!mx_plan(g, 0) || !mx_plan(d, 1) || gate.expert_bytes != up.expert_bytes) return MOE_ERR_UNSUPPORTED;
+  if (!mx_launch_args(*dims, T, gate, up, down, offsets, y_perm, ws, L)) return MOE_ERR_UNSUPPORTED;
+  const int H = dims->hidden, I = dims->inter;
   // the activations of every pair, in expert order, as E4M3 terms
-  const int64_t n8 = pairs * H / 8;
+  const int64_t n8 = L.pairs * H / 8;
   gather_split_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
-      static_cast<const uint4*>(x), perm, dims->top_k, H, pairs, kXTerms, xq, xs);
+      static_cast<const uint4*>(x), perm, dims->top_k, H, L.pairs, kXTerms, L.xq, L.xs);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
-  if (!make_term_map(&xmap, xq, kXTerms * pairs, H) || !make_term_map(&hmap, hq, kHTerms * pairs, I))
+  if (!make_term_map(&xmap, L.xq, kXTerms * L.pairs, H) || !make_term_map(&hmap, L.hq, kHTerms * L.pairs, I))
     return MOE_ERR_CUDA;
-  if ((st = launch_mx<0>(xmap, g, s)) != MOE_OK) return st;
-  return launch_mx<1>(hmap, d, s);
+  if ((st = launch_mx<0>(xmap, L.g, s)) != MOE_OK) return st;
+  return launch_mx<1>(hmap, L.d, s);
 }
 
 moe_status expert_gemm_dequant(const moe_dims* dims, const void* x, int32_t T, const moe_mxfp4_proj& gate,
                                const moe_mxfp4_proj& up, const moe_mxfp4_proj& down, const int32_t* offsets,
                                const int32_t* perm, float* y_perm, void* ws, cudaStream_t s) {
+  TcLaunch L;
+  // shape check before anything is enqueued
+  if (!tc_launch_args(*dims, T, gate, up, down, offsets, y_perm, ws, L)) return MOE_ERR_UNSUPPORTED;
   const int H = dims->hidden, I = dims->inter;
-  if (H % 64 || I % 64) return MOE_ERR_UNSUPPORTED;
-  const int64_t pairs = (int64_t)T * dims->top_k;
-  __half* x16 = static_cast<__half*>(ws);
-  __half* h16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + round_up((size_t)pairs * H * 2, 256));
-  TcArgs g{};
-  g.w0 = gate.base;
-  g.w1 = up.base;
-  g.expert_bytes = gate.expert_bytes;
-  g.rows = I;
-  g.a_cols = H;
-  g.k_total = H;
-  g.b_cols = H;
-  g.offsets = offsets;
-  g.E = dims->n_experts;
-  g.n_chunk = expert_chunk(T, dims->top_k, dims->n_experts);
-  g.out = h16;
-  g.limit = dims->swiglu_limit;
-  TcArgs d = g;
-  d.w0 = down.base;
-  d.w1 = nullptr;
-  d.expert_bytes = down.expert_bytes;
-  d.rows = H;
-  d.a_cols = I;
-  d.k_total = I;
-  d.b_cols = I;
-  d.out = y_perm;
-  {  // shape check before anything is enqueued
-    TcArgs pg = g, pd = d;
-    if (!tc_plan(pg, kAMxfp4) || !tc_plan(pd, kAMxfp4)) return MOE_ERR_UNSUPPORTED;
-  }
   // the activations of every pair, in expert order and f16 (the token operand
   // of the gate/up GEMM is then read with plain TMA boxes)
-  const int64_t n8 = pairs * H / 8;
+  const int64_t n8 = L.pairs * H / 8;
   gather_f16_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
-      static_cast<const uint4*>(x), perm, dims->top_k, H / 8, pairs, reinterpret_cast<uint4*>(x16));
+      static_cast<const uint4*>(x), perm, dims->top_k, H / 8, L.pairs, reinterpret_cast<uint4*>(L.x16));
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
-  if (!make_row_map(&xmap, x16, pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_row_map(&hmap, h16, pairs, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+  if (!make_row_map(&xmap, L.x16, L.pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_row_map(&hmap, L.h16, L.pairs, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
-  if ((st = launch_tc<0, kAMxfp4>(xmap, g, s)) != MOE_OK) return st;
-  return launch_tc<1, kAMxfp4>(hmap, d, s);
+  if ((st = launch_tc<0, kAMxfp4>(xmap, L.g, s)) != MOE_OK) return st;
+  return launch_tc<1, kAMxfp4>(hmap, L.d, s);
 }
 
 }  // namespace

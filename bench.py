@@ -168,10 +168,10 @@ def oracle_sample(dims, seed, layer, x_bits, router, bias, shared, tok=None, tab
     return blobs
 
 
-def time_oracle(dims, x_bits, router, bias, blobs, shared, tok=None, table=None):
+def time_oracle(dims, x_bits, router, bias, blobs, shared, tok=None, table=None, nthreads=None):
     """Seconds of one fp64 oracle pass over x_bits, the threads it used, its output."""
     import oracle
-    nthreads = os.cpu_count() or 1
+    nthreads = nthreads or os.cpu_count() or 1
     t0 = time.perf_counter()
     out, _, _ = oracle.moe_layer(dims, x_bits, np.arange(x_bits.shape[0]), router, bias, *blobs, shared=shared,
                                  tok=tok, table=table, nthreads=nthreads)
@@ -527,6 +527,11 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
                                         lay.table_np)
         cpu = {"value": n_tok / dt, "unit": unit, "cores": threads, "kind": "oracle",
                "sample": f"{n_tok} tokens of the batch-{B} layer (x set 0), whole layer in fp64"}
+        # the same oracle on one core, first token of the sample
+        dt1, _, _ = time_oracle(dims, xs[:1], lay.router_np, lay.bias_np, blobs, lay.shared_np,
+                                None if tok is None else tok[:1], lay.table_np, nthreads=1)
+        cpu["value_1_core"] = 1.0 / dt1
+        cpu["sample_1_core"] = "first token of the sample, 1 thread"
         # the same sample through the CUDA layer (untimed), against the oracle's
         # output; a failure here is reported in the line, not fatal to it
         try:

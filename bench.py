@@ -3,17 +3,22 @@
 
 Default workload (one "step"): one layer pass at each decode batch size
 1, 8, 32 and 64 tokens, each batch on its own resident layer (4 layers,
-13.9 GB of weights), with the token batch rotating over 4 seeded X sets so the
+13.7 GB of weights), with the token batch rotating over 4 seeded X sets so the
 routing changes from step to step.  A step streams ~5 GB of distinct expert
 weights, far above the 126 MB L2, so nothing is served from L2 across steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
-                    [--workload decode|prefill|hash|stack8|tiny]
+                    [--workload decode|decode64|prefill|hash|stack8|tiny] [--no-extra]
 
-Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs the same
-workload on its own GPU with its own weights (replicas, no collective on the
-data path); the time is the max over ranks and the value counts all ranks'
-tokens ("scaling": "weak").
+Prints one JSON line (rank 0).  The default decode run also measures the other
+four configurations (prefill T 4096, hash T 2048, 8 stacked layers at batch 32
+with a Zipf bias, the tiny layer) with a few timed steps each and reports them
+under "workloads": tokens/s, the dominant kernel's roofline fraction and an
+oracle parity sample for each.
+
+Multi-GPU (torchrun): every rank runs the same workload on its own GPU with its
+own weights (replicas, no collective on the data path); the time is the max
+over ranks and the value counts all ranks' tokens ("scaling": "weak").
 """
 from __future__ import annotations
 
@@ -34,7 +39,8 @@ sys.path.insert(0, ROOT)
 
 import gen  # noqa: E402
 
-EXPERT_BYTES = 3 * 4_456_448  # gate + up + down of one V4 expert
+METRIC = "MoE-layer tokens/s at V4-Flash shape; decode expert-weight HBM GB/s vs peak"
+UNIT = "tokens/s"
 
 
 # ---------------------------------------------------------------------------------------
@@ -57,6 +63,9 @@ def workload_spec(name):
     if name == "tiny":
         return gen.TINY, [(8, 0)], 4, "tiny_h256_e16_k2_t8"
     raise SystemExit(f"unknown workload {name}")
+
+
+EXTRA_WORKLOADS = ("prefill", "hash", "stack8", "tiny")
 
 
 def zipf_kappa():
@@ -96,61 +105,102 @@ class Layer:
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------------------
 
-class ClockSampler:
-    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, bus_id):
-        self.bus_id = bus_id
-        self.proc = None
-        self.lines = []
+
+class ClockSampler:
+    """SM clock, max clock and clock-event reasons of one GPU, sampled by a
+    thread through NVML every ~2 ms (through nvidia-smi every 50 ms if NVML
+    cannot be used)."""
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.rows = []  # (time, sm_mhz, max_mhz, [reason names])
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+        self.source = None
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
-        if self.bus_id:
-            cmd.insert(1, f"--id={self.bus_id}")
         try:
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.reader = threading.Thread(target=self._read, daemon=True)
-            self.reader.start()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else pynvml.nvmlDeviceGetHandleByIndex(0)
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            def loop():
+                while not self._stop.is_set():
+                    t = time.time()
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((t, float(sm), float(mx), [n for n, b in bits.items() if r & b]))
+                    except Exception:  # noqa: BLE001
+                        pass
+                    time.sleep(0.002)
+
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml, ~2 ms"
+        except Exception:  # noqa: BLE001
+            self._start_smi()
+
+    def _start_smi(self):
+        fields = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        cmd = ["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.uuid:
+            cmd.insert(1, f"--id={self.uuid}")
+        try:
+            self._proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+
+        def read():
+            for line in self._proc.stdout:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    self.rows.append((time.time(), float(f[1]), float(f[2]),
+                                      [REASON_NAMES[i] for i in range(4) if f[5 + i].lower() == "active"]))
+                except ValueError:
+                    continue
+
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
+        self.source = "nvidia-smi, 50 ms"
 
     def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        rows = []
-        for ts, line in self.lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append((ts, float(f[1]), float(f[2]), f[5:9]))
-            except ValueError:
-                continue
-        inside = [r for r in rows if t0 <= r[0] <= t1]
-        window = inside if inside else [r for r in rows if t0 - 0.25 <= r[0] <= t1 + 0.25]
+        inside = [r for r in self.rows if t0 <= r[0] <= t1]
+        window = inside if inside else [r for r in self.rows if t0 - 0.25 <= r[0] <= t1 + 0.25]
         if not window:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in window for i in range(4) if r[3][i].lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = sorted({n for r in window for n in r[3]})
         return {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": max(r[2] for r in window),
-                "reasons": reasons, "samples": len(window), "samples_inside_timed_region": len(inside)}
+                "reasons": reasons, "samples": len(window), "samples_inside_timed_region": len(inside),
+                "source": self.source}
 
 
 # ---------------------------------------------------------------------------------------
-# the oracle on the host cores (cpu_baseline and --impl reference)
+# the oracle on the host cores (cpu_baseline, parity samples and --impl reference)
 # ---------------------------------------------------------------------------------------
 
 def oracle_sample(dims, seed, layer, x_bits, router, bias, shared, tok=None, table=None):
@@ -185,13 +235,6 @@ def parity_stats(got, want):
     want = np.asarray(want, np.float64)
     err = np.abs(got - want)
     return float(err.max() / np.sqrt(np.mean(want ** 2))), float(err.sum() / np.abs(want).sum())
-
-
-def sample_inputs(dims, spec_batches, seed, n_tok):
-    """The first n_tok tokens of x set 0 of the last batch of the workload."""
-    B, layer = spec_batches[-1]
-    x = gen.x_rows(seed, layer, min(n_tok, B), dims.hidden)
-    return x, layer
 
 
 def run_reference(args, dims, batches, desc, metric, unit):
@@ -235,13 +278,17 @@ def run_reference(args, dims, batches, desc, metric, unit):
 SPEC_HBM_GBS = 8000.0
 SPEC_BF16_TFLOPS = 2250.0
 
-# moe_expert_gemm runs the block-scaled kernel when an expert averages at most
-# 8 pairs (the library's path choice from T), else the dequantising kernel.
+# moe_expert_gemm's kernels by path (the library picks the path from T alone)
 EXPERT_KERNELS = {
     "block_scaled": ("mx_expert_kernel (moe_expert_gemm: block-scaled tcgen05 mxf8f6f4, gate/up+SwiGLU and down)",
                      ("mx_expert.cuh", "tc_expert.cuh", "common.cuh")),
     "dequant": ("tc_expert_kernel (moe_expert_gemm: E2M1 dequantised to f16, tcgen05 f16, gate/up+SwiGLU and down)",
                 ("tc_expert.cuh", "common.cuh")),
+}
+# the arithmetic each path computes in
+EXPERT_DTYPES = {
+    "block_scaled": "mxfp4 x e4m3 (x as 2 terms, h as 3 terms), f32 accumulate",
+    "dequant": "mxfp4 dequantised to f16 x f16, f32 accumulate",
 }
 
 
@@ -283,36 +330,36 @@ def whole_job_rate(world, units_per_step_per_rank, steps, seconds):
     return world * units_per_step_per_rank * steps / seconds
 
 
-def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
-    import torch
+def load_peaks():
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    return json.load(open(pk)) if os.path.exists(pk) else {}
 
-    import __graft_entry__
-    import mxfp4_routed_expert_sqrt_b200 as m
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
+class Ctx:
+    """Process-wide state of one bench run."""
 
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if rank == 0:
-        __graft_entry__.build()
-    if dist is not None:
-        dist.barrier()
-    m.lib()
+    def __init__(self, torch, m, dist, dev, rank, world):
+        self.torch, self.m, self.dist, self.dev, self.rank, self.world = torch, m, dist, dev, rank, world
+        self.peaks = load_peaks()
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:  # noqa: BLE001
+            self.uuid = None
 
+
+def measure(ctx, workload, steps, warmup, full=True, no_cpu_baseline=False):
+    """Times `steps` steps of a workload (after `warmup`), returns its record.
+
+    full: also the e2e leg, the 1-core oracle figure and the clocks (the
+    headline workload); otherwise a compact record for the workloads object."""
+    torch, m, dist, dev, rank, world = ctx.torch, ctx.m, ctx.dist, ctx.dev, ctx.rank, ctx.world
+    dims, batches, n_xsets, desc = workload_spec(workload)
     seed = 0
-    H, K = dims.hidden, dims.top_k
-    hashed = args.workload == "hash"
+    H, K, I = dims.hidden, dims.top_k, dims.inter
+    hashed = workload == "hash"
     bias = None
     kappa = None
-    if args.workload == "stack8":
+    if workload == "stack8":
         kappa = zipf_kappa()
         if kappa is None:
             raise SystemExit("stack8 needs tests/golden/zipf_kappa.json (tests/golden/make_zipf_kappa.py)")
@@ -323,8 +370,7 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
             layers[l] = Layer(m, torch, dims, seed, l, dev, hashed=hashed, bias=bias)
     # x sets: seed shifted per set and rank, so ranks and steps route differently
     t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev).view(dt)
-    xsets = {}
-    toksets = {}
+    xsets, toksets = {}, {}
     for j, (B, l) in enumerate(batches):
         for s in range(n_xsets):
             xs = gen.x_rows(seed + 1000 * (s + 1) + 100000 * rank, l, B, H)
@@ -353,35 +399,47 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         # implementation detail, not counted.
         B = batches[j][0]
         U = distinct[(j, s)]
-        I = dims.inter
         act = B * H * 2 + 2 * B * K * I * 2 + B * K * H * 4
         return U * (3 * (I * H // 2 + I * H // 32)) + act
 
+    def layer_bytes(j, s):
+        # whole layer: expert call + shared expert (bf16, 3 I H) + router (fp32, E H)
+        # + x read by route and shared, out written (fp32), combine's y_perm read
+        B = batches[j][0]
+        return (expert_bytes(j, s) + 3 * I * H * 2 + dims.n_experts * H * 4 + 2 * B * H * 2 + B * H * 4
+                + B * K * H * 4)
+
     # route 2 (3 with the tensor-core router split), permute 1, shared 2,
     # experts 3 (activation gather, gate/up, down), combine 1
-    n_layer_kernels = 9 + (1 if batches[0][0] > 64 and dims.n_experts % 256 == 0 else 0)
+    def kernels_of(B):
+        return 9 + (1 if B > 64 and dims.n_experts % 256 == 0 else 0)
 
     def one_step(i, events=None):
         s = i % n_xsets
         for j, (B, l) in enumerate(batches):
             ev = None if events is None else events[j]
+            if ev is not None:
+                ev[2].record()
             runners[j].forward(layers[l].w, xsets[(j, s)][1], B, outs[j], token_ids=toksets.get((j, s)),
-                               expert_events=ev)
+                               expert_events=None if ev is None else ev[:2])
+            if ev is not None:
+                ev[3].record()
 
-    # graphs: the timed steps are captured in chunks, each (step, batch) with its own event pair
+    # graphs: the timed steps are captured in chunks, each (step, batch) with
+    # event pairs around its routed-expert call and around the whole layer
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
-    chunk = max(1, min(args.steps, 10))
+    chunk = max(1, min(steps, 10))
     warm_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(warm_graph, stream=stream):
         for i in range(n_xsets):
             one_step(i)
     timed = []
     step = 0
-    while step < args.steps:
-        n = min(chunk, args.steps - step)
-        evs = [[(torch.cuda.Event(enable_timing=True, external=True),
-                 torch.cuda.Event(enable_timing=True, external=True)) for _ in batches] for _ in range(n)]
+    while step < steps:
+        n = min(chunk, steps - step)
+        evs = [[tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)) for _ in batches]
+               for _ in range(n)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
@@ -391,22 +449,18 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     torch.cuda.synchronize()
 
     # warm-up: W steps (replays of the n_xsets-step graph, rounded up)
-    for _ in range(max(1, (args.warmup + n_xsets - 1) // n_xsets)):
+    for _ in range(max(1, (warmup + n_xsets - 1) // n_xsets)):
         warm_graph.replay()
     torch.cuda.synchronize()
 
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        gpu_id = None
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
-    # pre-roll so the clocks and the sampler are live when timing starts
-    t_pre = time.time()
-    while time.time() - t_pre < 0.4:
-        warm_graph.replay()
-        torch.cuda.synchronize()
+    sampler = ClockSampler(ctx.uuid) if full else None
+    if sampler is not None:
+        sampler.start()
+        # pre-roll so the clocks and the sampler are live when timing starts
+        t_pre = time.time()
+        while time.time() - t_pre < 0.3:
+            warm_graph.replay()
+            torch.cuda.synchronize()
 
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -425,40 +479,42 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
     wall1 = time.time()
     if dist is not None:
         dist.barrier()
-    # keep the GPU busy a little longer so the sampler brackets the region
-    t_post = time.time()
-    while time.time() - t_post < 0.2:
-        warm_graph.replay()
-        torch.cuda.synchronize()
-    sampler.stop()
+    if sampler is not None:
+        sampler.stop()
     ms = max_over_ranks(dist, ev0.elapsed_time(ev1), dev)
     tokens_per_step = sum(B for B, _ in batches)
-    value = whole_job_rate(world, tokens_per_step, args.steps, ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, steps, ms / 1e3)
 
-    # roofline of the routed-expert GEMV (moe_expert_gemm: gate/up and down launches)
-    k_ms, k_bytes, n_calls = 0.0, 0, 0
+    # the routed-expert call (moe_expert_gemm: activation gather, gate/up and
+    # down launches), per batch position and over all calls
+    per = {j: {"k_ms": 0.0, "k_bytes": 0, "l_ms": 0.0, "l_bytes": 0, "n": 0, "U": 0} for j in range(len(batches))}
     for g, s0, n, evs in timed:
         for i in range(n):
             for j in range(len(batches)):
-                a, b = evs[i][j]
-                k_ms += a.elapsed_time(b)
-                k_bytes += expert_bytes(j, (s0 + i) % n_xsets)
-                n_calls += 1
-    import json as _json
-    peaks = {}
-    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(pk):
-        peaks = _json.load(open(pk))
+                a, b, c, d = evs[i][j]
+                s = (s0 + i) % n_xsets
+                per[j]["k_ms"] += a.elapsed_time(b)
+                per[j]["k_bytes"] += expert_bytes(j, s)
+                per[j]["l_ms"] += c.elapsed_time(d)
+                per[j]["l_bytes"] += layer_bytes(j, s)
+                per[j]["U"] += distinct[(j, s)]
+                per[j]["n"] += 1
+    k_ms = sum(p["k_ms"] for p in per.values())
+    k_bytes = sum(p["k_bytes"] for p in per.values())
+    n_calls = sum(p["n"] for p in per.values())
+    peaks = ctx.peaks
     path = expert_path(dims, batches[0][0])
     assert all(expert_path(dims, B) == path for B, _ in batches)
     traffic = traffic_record(desc, path)
     kernel = EXPERT_KERNELS[path][0]
-    if args.workload == "prefill":
+    hbm_peak = peaks.get("hbm_gbs") or 6650.0
+    hbm_src = "measured" if peaks.get("hbm_gbs") else "fallback"
+    if workload == "prefill":
         # tensor bound (~96 pairs per expert, arithmetic intensity above the ridge):
-        # algorithmic flops = pairs * 3 projections * 2 * H * I (f16 x f16, same
-        # nominal rate as bf16); the GEMM runs inside a multi-millisecond step.
+        # algorithmic flops = pairs * 3 projections * 2 * H * I; the GEMM runs
+        # inside a multi-millisecond step, so the sustained bf16 peak applies.
         # The hash workload (~48 pairs per expert) sits below the ridge: HBM bound.
-        flops = sum(B * K * 3 * 2 * H * dims.inter for B, _ in batches) * args.steps
+        flops = sum(B * K * 3 * 2 * H * I for B, _ in batches) * steps
         peak = peaks.get("bf16_tflops_sustained")
         peak_src = "measured sustained bf16" if peak else "fallback sustained"
         peak = peak or 1400.0
@@ -469,80 +525,90 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
                     "kernel": kernel, "algorithmic_flops_per_launch": int(flops / n_calls),
                     "avg_launch_ms": round(k_ms / n_calls, 5)}
     else:
-        peak = peaks.get("hbm_gbs")
-        peak_src = "measured" if peak else "fallback"
-        peak = peak or 6650.0
         achieved = k_bytes / (k_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                    "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "peak_source": hbm_src,
                     "spec_peak": SPEC_HBM_GBS, "frac_spec": round(achieved / SPEC_HBM_GBS, 4),
                     "kernel": kernel, "algorithmic_bytes_per_launch": int(k_bytes / n_calls),
                     "avg_launch_ms": round(k_ms / n_calls, 5)}
-
-    # e2e: the public API with pinned host buffers, H2D + layer + D2H every step
-    h_in = []
-    h_out = []
-    graphs_e2e = []
+    l_bytes = sum(p["l_bytes"] for p in per.values())
+    l_ms = sum(p["l_ms"] for p in per.values())
+    roofline["whole_layer_gbs"] = round(l_bytes / (l_ms / 1e3) / 1e9, 1)
+    roofline["whole_layer_frac"] = round(l_bytes / (l_ms / 1e3) / 1e9 / hbm_peak, 4)
+    per_batch = []
     for j, (B, l) in enumerate(batches):
-        hx = torch.empty(B * H, dtype=torch.bfloat16, pin_memory=True)
-        hx.copy_(xsets[(j, 0)][1].view(-1).cpu())
-        ho = torch.empty(B * H, dtype=torch.float32, pin_memory=True)
-        h_in.append(hx)
-        h_out.append(ho)
-        graphs_e2e.append(runners[j].graphed(layers[l].w, B, hx, ho, token_ids=toksets.get((j, 0)), stream=stream))
-    for _ in range(2):
-        for ge in graphs_e2e:
-            ge()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    # device-timed on the replay stream; each step waits for its result on the
-    # host, so the region holds the copies, the layer and the host round trip
-    ev_e0, ev_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev_e0.record(stream)
-    for _ in range(args.steps):
-        for ge in graphs_e2e:
-            ge()
-        stream.synchronize()
-    ev_e1.record(stream)
-    ev_e1.synchronize()
-    e2e_s = max_over_ranks(dist, ev_e0.elapsed_time(ev_e1) / 1e3, dev)
-    e2e = {"value": whole_job_rate(world, tokens_per_step, args.steps, e2e_s), "unit": unit,
-           "h2d_bytes_per_step": sum(B * H * 2 for B, _ in batches),
-           "d2h_bytes_per_step": sum(B * H * 4 for B, _ in batches)}
+        p = per[j]
+        gbs = p["k_bytes"] / (p["k_ms"] / 1e3) / 1e9
+        per_batch.append({"batch": B, "layer": l, "distinct_experts": round(p["U"] / p["n"], 1),
+                          "expert_call_us": round(1e3 * p["k_ms"] / p["n"], 2), "expert_call_gbs": round(gbs, 1),
+                          "expert_call_frac": round(gbs / hbm_peak, 4),
+                          "layer_us": round(1e3 * p["l_ms"] / p["n"], 2),
+                          "layer_tokens_per_s": round(B * p["n"] / (p["l_ms"] / 1e3), 1)})
+
+    e2e = None
+    if full:
+        # e2e: the public API with pinned host buffers, H2D + layer + D2H every step
+        graphs_e2e = []
+        for j, (B, l) in enumerate(batches):
+            hx = torch.empty(B * H, dtype=torch.bfloat16, pin_memory=True)
+            hx.copy_(xsets[(j, 0)][1].view(-1).cpu())
+            ho = torch.empty(B * H, dtype=torch.float32, pin_memory=True)
+            graphs_e2e.append(runners[j].graphed(layers[l].w, B, hx, ho, token_ids=toksets.get((j, 0)),
+                                                 stream=stream))
+        for _ in range(2):
+            for ge in graphs_e2e:
+                ge()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        # device-timed on the replay stream; each step waits for its result on the
+        # host, so the region holds the copies, the layer and the host round trip
+        ev_e0, ev_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_e0.record(stream)
+        for _ in range(steps):
+            for ge in graphs_e2e:
+                ge()
+            stream.synchronize()
+        ev_e1.record(stream)
+        ev_e1.synchronize()
+        e2e_s = max_over_ranks(dist, ev_e0.elapsed_time(ev_e1) / 1e3, dev)
+        e2e = {"value": whole_job_rate(world, tokens_per_step, steps, e2e_s), "unit": UNIT,
+               "h2d_bytes_per_step": sum(B * H * 2 for B, _ in batches),
+               "d2h_bytes_per_step": sum(B * H * 4 for B, _ in batches)}
+        del graphs_e2e
     assert m.moe_device_error() == 0
 
+    # the oracle: cpu_baseline (headline only) and a parity sample of the layer
     cpu = None
     parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok = 8 if args.workload != "tiny" else 8
+    if rank == 0 and world == 1 and not no_cpu_baseline:
+        n_tok = 8 if full else 2
         B, l = batches[-1]
-        xs = xsets[(len(batches) - 1, 0)][0][:n_tok]
+        jl = len(batches) - 1
+        xs = xsets[(jl, 0)][0][:n_tok]
         lay = layers[l]
-        tok = None
-        if hashed:
-            tok = toksets[(len(batches) - 1, 0)].cpu().numpy()[:n_tok]
+        tok = toksets[(jl, 0)].cpu().numpy()[:n_tok] if hashed else None
         blobs = oracle_sample(dims, seed, l, xs, lay.router_np, lay.bias_np, lay.shared_np, tok, lay.table_np)
         dt, threads, want = time_oracle(dims, xs, lay.router_np, lay.bias_np, blobs, lay.shared_np, tok,
                                         lay.table_np)
-        cpu = {"value": n_tok / dt, "unit": unit, "cores": threads, "kind": "oracle",
-               "sample": f"{n_tok} tokens of the batch-{B} layer (x set 0), whole layer in fp64"}
-        # the same oracle on one core, first token of the sample
-        dt1, _, _ = time_oracle(dims, xs[:1], lay.router_np, lay.bias_np, blobs, lay.shared_np,
-                                None if tok is None else tok[:1], lay.table_np, nthreads=1)
-        cpu["value_1_core"] = 1.0 / dt1
-        cpu["sample_1_core"] = "first token of the sample, 1 thread"
+        sample = f"{n_tok} tokens of the batch-{B} layer (x set 0), whole layer in fp64"
+        if full:
+            cpu = {"value": n_tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+            # the same oracle on one core, first token of the sample
+            dt1, _, _ = time_oracle(dims, xs[:1], lay.router_np, lay.bias_np, blobs, lay.shared_np,
+                                    None if tok is None else tok[:1], lay.table_np, nthreads=1)
+            cpu["value_1_core"] = 1.0 / dt1
+            cpu["sample_1_core"] = "first token of the sample, 1 thread"
         # the same sample through the CUDA layer (untimed), against the oracle's
         # output; a failure here is reported in the line, not fatal to it
         try:
-            jl = len(batches) - 1
             out_s = torch.empty(n_tok * H, dtype=torch.float32, device=dev)
             runners[jl].forward(lay.w, xsets[(jl, 0)][1][:n_tok], n_tok, out_s,
                                 token_ids=toksets[(jl, 0)][:n_tok] if hashed else None)
             torch.cuda.synchronize()
             dev_err = m.moe_device_error()
             mx_err, l1_err = parity_stats(out_s.view(n_tok, H).cpu().numpy(), want)
-            parity = {"sample": cpu["sample"], "max_err_over_rms": mx_err, "sum_err_over_sum_ref": l1_err,
+            parity = {"sample": sample, "max_err_over_rms": mx_err, "sum_err_over_sum_ref": l1_err,
                       "tolerance": {"max_err_over_rms": 1e-2, "sum_err_over_sum_ref": 2e-3},
                       "device_error": dev_err}
             if not hashed:  # the bench's x sets are not redrawn: how close routing came to a tie
@@ -553,26 +619,79 @@ def run_mine(args, dims, batches, n_xsets, desc, metric, unit):
         except Exception as exc:  # noqa: BLE001
             parity = {"error": repr(exc)[:300]}
 
-    clocks = sampler.summary(wall0, wall1)
+    clocks = sampler.summary(wall0, wall1) if sampler is not None else None
+    rec = {"workload": desc, "value": value, "ms_per_step": ms / steps, "steps": steps, "warmup": warmup,
+           "tokens_per_step": tokens_per_step, "batches": [B for B, _ in batches], "roofline": roofline,
+           "per_batch": per_batch, "parity": parity, "path": path, "dtype": EXPERT_DTYPES[path],
+           "gpu_launches": sum(kernels_of(B) for B, _ in batches) * steps, "zipf_kappa": kappa,
+           "dims": {"hidden": H, "inter": I, "experts": dims.n_experts, "top_k": K}}
+    if full:
+        rec.update({"e2e": e2e, "cpu_baseline": cpu, "clocks": clocks})
     for g, _, _, _ in timed:
         del g
+    del timed, warm_graph, layers, runners, outs, xsets, toksets
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_mine(args):
+    import torch
+
+    import __graft_entry__
+    import mxfp4_routed_expert_sqrt_b200 as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
     if rank == 0:
-        line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": {"workload": desc, "hidden": dims.hidden, "inter": dims.inter,
-                           "experts": dims.n_experts, "top_k": dims.top_k,
-                           "batches": [B for B, _ in batches], "tokens_per_step": tokens_per_step,
+        __graft_entry__.build()
+    if dist is not None:
+        dist.barrier()
+    m.lib()
+    ctx = Ctx(torch, m, dist, dev, rank, world)
+
+    head = measure(ctx, args.workload, args.steps, args.warmup, full=True, no_cpu_baseline=args.no_cpu_baseline)
+    extra = {}
+    if args.workload == "decode" and not args.no_extra:
+        # the other configurations, a few timed steps each (device-timed the same way)
+        for w in EXTRA_WORKLOADS:
+            r = measure(ctx, w, max(3, min(args.steps, 10)), 3, full=False, no_cpu_baseline=args.no_cpu_baseline)
+            extra[w] = {k: r[k] for k in ("workload", "value", "ms_per_step", "steps", "tokens_per_step", "path",
+                                          "dtype", "parity")}
+            extra[w]["unit"] = UNIT
+            extra[w]["roofline"] = {k: r["roofline"].get(k) for k in
+                                    ("bound", "achieved", "peak", "unit", "frac", "frac_spec", "kernel",
+                                     "avg_launch_ms", "traffic", "whole_layer_gbs")}
+            if w == "stack8":
+                extra[w]["zipf_kappa"] = r["zipf_kappa"]
+                extra[w]["per_layer_expert_gbs"] = [p["expert_call_gbs"] for p in r["per_batch"]]
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic",
+                "config": {"workload": head["workload"], **head["dims"], "batches": head["batches"],
+                           "tokens_per_step": head["tokens_per_step"],
                            "weights": "mxfp4 (e2m1 + e8m0/32), shared expert bf16, router fp32",
-                           "accumulate": "f32", "parallelism": f"replicas x{world}",
+                           "expert_path": head["path"], "parallelism": f"replicas x{world}",
                            "l2": "inputs larger than L2: each step streams distinct expert weights "
                                  "of resident layers (no flush)",
-                           "cuda_graphs": True, "zipf_kappa": kappa},
-                "roofline": roofline, "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
-                "gpu_launches": n_layer_kernels * len(batches) * args.steps,
-                "clocks": clocks}
+                           "cuda_graphs": True, "zipf_kappa": head["zipf_kappa"]},
+                "roofline": head["roofline"], "per_batch": head["per_batch"], "cpu_baseline": head["cpu_baseline"],
+                "parity": head["parity"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+                "clocks": head["clocks"]}
+        if extra:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
-    del timed, warm_graph, graphs_e2e
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -586,16 +705,15 @@ def main():
     ap.add_argument("--impl", choices=("mine", "reference"), default="mine")
     ap.add_argument("--workload", default="decode", choices=("decode", "decode64", "prefill", "hash", "stack8", "tiny"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="decode only: skip the other four configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     dims, batches, n_xsets, desc = workload_spec(args.workload)
-    metric = "MoE-layer tokens/s at V4-Flash shape; decode expert-weight HBM GB/s vs peak"
-    unit = "tokens/s"
     if args.impl == "reference":
-        run_reference(args, dims, batches, desc, metric, unit)
+        run_reference(args, dims, batches, desc, METRIC, UNIT)
     else:
-        run_mine(args, dims, batches, n_xsets, desc, metric, unit)
+        run_mine(args)
 
 
 if __name__ == "__main__":

@@ -89,10 +89,16 @@ int moe_abi_version(void);
 const char* moe_status_string(moe_status status);
 
 /* Reads and clears the device error word of the current device (host call,
- * synchronises the current device).  0 = no error; otherwise a code naming
- * the kernel that gave up a bounded wait: 0x201 an expert id outside [0, E)
- * reached moe_permute, 0x301 a tensor-core kernel gave up waiting on a copy
- * (each wait is bounded to 2 s), 0x401 moe_selftest_wait. */
+ * synchronises the current device).  0 = no error; otherwise the first code
+ * recorded since the last read:
+ *   0x201  an expert id outside [0, E) reached moe_permute;
+ *   0x301  a tensor-core kernel gave up waiting on a copy (each wait is
+ *          bounded to 2 s);
+ *   0x302  moe_expert_gemm's dequantising path met a weight row whose E8M0
+ *          bytes span more than 36 octaves and flushed its lowest groups;
+ *   0x303  moe_expert_gemm's dequantising path met an activation beyond the
+ *          f16 range (|x| > 65504); that call's output is undefined;
+ *   0x401  moe_selftest_wait. */
 int32_t moe_device_error(void);
 
 /* Health check of the bounded-wait path (no counterpart on the pages): a
@@ -150,6 +156,9 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
  *  - The array keeps the previous call's logits; every call overwrites the
  *    T * n_experts entries it reads before reading them, so nothing has to
  *    start at zero.
+ *  - The looked-up address is kept per device and driver context; a new
+ *    context on a device (after cudaDeviceReset, say) is looked up again
+ *    on its first call.
  * Arguments and outputs are those of moe_route (no ws / ws_bytes).
  * No device memory is allocated or freed by this call.
  */
@@ -201,12 +210,17 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *    Workspace: E4M3 terms and E8M0 scales of x in expert order
  *    [2][T*top_k][hidden] and [2][T*top_k][hidden/32], then of h
  *    [3][T*top_k][inter] and [3][T*top_k][inter/32] bytes.
- *  - above 8 (prefill): each weight is dequantised exactly to f16 (up to a
- *    power of two per row undone in fp32) as long as the E8M0 exponents of
- *    one weight row span at most 36 octaves; x goes in as f16 (|x| below
- *    65504, values under 2^-14 keep f16 subnormal precision), h between the
- *    GEMMs is f16; f16 x f16 MMAs with fp32 sums.  Workspace: x in expert
- *    order as f16 [T*top_k][hidden], then h in f16 [T*top_k][inter].
+ *  - above 8 (prefill): each weight is dequantised to f16 times a power of
+ *    two per weight row (undone in fp32): exactly for every E8M0 group within
+ *    36 octaves of the largest group of its row, whatever the bytes; groups
+ *    further below are flushed to zero (their products lie below 2^-36 of
+ *    the row's largest group's) and the call records device error 0x302.
+ *    x goes in as f16: exact for |x| in [2^-17, 65504], f16 subnormal
+ *    precision below (absolute error at most 2^-25); a value beyond 65504
+ *    is not representable and the call records device error 0x303 (its
+ *    output is undefined).  h between the GEMMs is f16; f16 x f16 MMAs with
+ *    fp32 sums.  Workspace: x in expert order as f16 [T*top_k][hidden], then
+ *    h in f16 [T*top_k][inter].
  * Shapes: inter a multiple of 128, hidden a multiple of 256 (the row tiles of
  * the two GEMMs), besides the moe_dims limits; other shapes return
  * MOE_ERR_UNSUPPORTED before anything is enqueued.

@@ -139,6 +139,8 @@ def moe_device_error() -> int:
 # device error codes (moe_device_error)
 DEVICE_ERR_BAD_EXPERT = 0x201
 DEVICE_ERR_WAIT_TC = 0x301
+DEVICE_ERR_SPAN_FLUSH = 0x302
+DEVICE_ERR_F16_RANGE = 0x303
 DEVICE_ERR_WAIT_SELFTEST = 0x401
 
 

@@ -17,6 +17,8 @@ enum : int32_t {
   kErrNone = 0,
   kErrBadExpert = 0x201,    // an expert id outside [0, E) reached moe_permute
   kErrWaitTc = 0x301,       // tensor-core kernel gave up waiting on an mbarrier
+  kErrSpanFlush = 0x302,    // a weight row's E8M0 bytes span > 36 octaves: the lowest groups were flushed
+  kErrF16Range = 0x303,     // an activation beyond the f16 range reached the dequantising expert path
   kErrWaitSelftest = 0x401, // moe_selftest_wait: its wait ran out, as it should
 };
 

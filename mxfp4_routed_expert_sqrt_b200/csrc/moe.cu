@@ -238,23 +238,53 @@ static __device__ __align__(256) float g_route_noalloc_logits[MOE_ROUTE_NOALLOC_
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-float* g_noalloc_ptr[kMaxDevices] = {};
+// Per device: the scratch array's device address and the context it was
+// looked up in.  A device reset (cudaDeviceReset) tears the context down and
+// the module is loaded again, possibly elsewhere; a new context on the same
+// device is the sign that the address has to be looked up again.
+struct NoallocSlot {
+  const void* ctx;
+  float* ptr;
+};
+NoallocSlot g_noalloc[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device; looked up once
-// per device (the host-side symbol is not a device address).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The current thread's driver context (through the runtime's entry point
+// table, so the library needs no libcuda link); null if unavailable.
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext c = nullptr;
+  return fn(&c) == CUDA_SUCCESS ? static_cast<void*>(c) : nullptr;
+}
+
+// Device address of the scratch array on the current device, looked up with
+// that device current the first time it is needed in a context (the host-side
+// symbol is not a device address).
 cudaError_t noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const void* ctx = current_context();  // null before the runtime has made one current
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc[dev];
+  if (slot.ptr == nullptr || ctx == nullptr || slot.ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_noalloc_logits);
+    e = cudaGetSymbolAddress(&p, g_route_noalloc_logits);  // makes the device's context current
     if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
+    slot.ptr = static_cast<float*>(p);
+    slot.ctx = current_context();
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 }  // namespace

@@ -10,10 +10,11 @@
 //   MODE 1 (down):     acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter, fp32 out
 // MXFP4 operands run as f16 x f16 MMAs (fp32 accumulation): activations come
 // in f16 and each weight is dequantised exactly to f16 as v * 2^(e - 127 -
-// c_r), c_r = max(0, e_max(row) - 140), with 2^c_r applied to the fp32
-// accumulator row in the epilogue.  That is exact whenever a row's E8M0
-// exponents span at most 36 octaves, and costs two instructions per pair of
-// codes (cvt + multiply).  bf16 weights (shared expert, router) are copied as
+// c_r), c_r = e_max(row) - 140 (signed), with 2^c_r applied to the fp32
+// accumulator row in the epilogue.  That is exact for every group within 36
+// octaves of its row's largest (any E8M0 byte otherwise); groups further below
+// are flushed to zero and the call records device error 0x302.  Two
+// instructions per pair of codes (cvt + multiply).  bf16 weights (shared expert, router) are copied as
 // they are.
 // ("Model techniques map", row "SwiGLU feed-forward": the clamped SwiGLU;
 // "ElytronAI / DeepSeek-v4-Flash", Sizes/Layout: MXFP4 weights, expert xid at
@@ -192,6 +193,20 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ uint32_t pow2_f16x2(int k) {
   const float f = __uint_as_float((uint32_t)(k + 127) << 23);
   return f32x2_to_f16x2(f, f);
+}
+
+// Octaves below a row's largest E8M0 group that still dequantise exactly: a
+// code v in {0.5, ..., 6} times 2^k is an f16 value (subnormals included) for
+// k in [-23, 13].
+constexpr int kF16Span = 36;
+
+// Dequantisation factor of one group, k = e - 127 - c_r <= 13: 2^k as f16x2,
+// or 0 (the group flushed) below the exact range.
+__device__ __forceinline__ uint32_t group_factor_f16x2(int k) { return k >= -23 ? pow2_f16x2(k) : 0u; }
+
+// 2^k as fp32 for k in [-149, 127] (subnormal below -126).
+__device__ __forceinline__ float pow2_f32(int k) {
+  return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << (k + 149));
 }
 
 // Byte offset inside a TMA box written with the swizzle mode that matches its
@@ -449,12 +464,25 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
           const int b = 4 * w;
           return *reinterpret_cast<const uint32_t*>(scb + (b / cs) * kTcAThreads * cs + b % cs);
         };
-        // per-row exponent offset keeping v * 2^(e-127-c_r) inside f16
-        uint32_t mx = 0;
-        for (int w = 0; w < sr / 4; ++w) mx = __vmaxu4(mx, sc_word(w));
+        // per-row exponent offset c_r = e_max(row) - 140 (signed): every group
+        // factor 2^(e-127-c_r) = 2^(e - e_max + 13) is at most 2^13, so the
+        // largest code (6) stays inside f16, and groups down to 36 octaves
+        // below the row's largest are exact f16 values
+        uint32_t mx = 0, mn = 0xFFFFFFFFu;
+        for (int w = 0; w < sr / 4; ++w) {
+          const uint32_t v = sc_word(w);
+          mx = __vmaxu4(mx, v);
+          mn = __vminu4(mn, v);
+        }
         mx = __vmaxu4(mx, mx >> 16);
         mx = __vmaxu4(mx, mx >> 8);
-        const int crow = max(0, (int)(mx & 0xFFu) - 140);
+        mn = __vminu4(mn, mn >> 16);
+        mn = __vminu4(mn, mn >> 8);
+        const int crow = (int)(mx & 0xFFu) - 140;
+        // a wider span cannot be exact in f16: those groups are flushed to
+        // zero (their products are below 2^-36 of the row's largest group's)
+        // and the call is flagged
+        if ((int)(mx & 0xFFu) - (int)(mn & 0xFFu) > kF16Span) set_error(kErrSpanFlush);
         s_crow[un % kCrowRing][t][r] = (int16_t)crow;
         // k-block g of the current stage of this row -> 64 f16 values
         auto convert = [&](int g, uint32_t sw, uint32_t (&v)[32]) {
@@ -464,8 +492,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
           const uint4 c1 = *reinterpret_cast<const uint4*>(tile + swz(o + 16, mask));
           const int e0 = (int)((sw >> (16 * g)) & 0xFFu), e1 = (int)((sw >> (16 * g + 8)) & 0xFFu);
           const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          const uint32_t f0 = pow2_f16x2(max(e0 - 127 - crow, -24));
-          const uint32_t f1 = pow2_f16x2(max(e1 - 127 - crow, -24));
+          const uint32_t f0 = group_factor_f16x2(e0 - 127 - crow);
+          const uint32_t f1 = group_factor_f16x2(e1 - 127 - crow);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t hv[4];
@@ -681,8 +709,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       // acc1), written before this unit's first stage
       float s0 = 1.f, s1 = 1.f;
       if (AF == kAMxfp4) {
-        s0 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][0][r] + 127) << 23);
-        s1 = __uint_as_float((uint32_t)(s_crow[un % kCrowRing][1][r] + 127) << 23);
+        s0 = pow2_f32(s_crow[un % kCrowRing][0][r]);
+        s1 = pow2_f32(s_crow[un % kCrowRing][1][r]);
       }
       for (int c0 = 16 * half; c0 < n; c0 += 16 * (EPI / 4)) {
         uint32_t g[16], h[16];
@@ -731,18 +759,28 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   }
 }
 
+// True when either half of an f16x2 is infinite.
+__device__ __forceinline__ bool f16x2_has_inf(uint32_t h) {
+  return (h & 0x7FFFu) == 0x7C00u || ((h >> 16) & 0x7FFFu) == 0x7C00u;
+}
+
 // Activations in pair order for the gate/up GEMM: out[pos] = f16(x[perm[pos] /
-// K]), rows of h8 groups of 8 values.  Exact for |x| in [2^-14, 65504], f16
-// subnormals below; |x| > 65504 is out of range.
+// K]), rows of h8 groups of 8 values.  Exact for |x| in [2^-17, 65504] (f16
+// subnormals carry bf16's 8 bits down to 2^-17); a value beyond 65504 becomes
+// inf and the call records device error 0x303.
 __global__ void gather_f16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int K, int h8,
                                   int64_t rows, uint4* __restrict__ out) {
   const int64_t n = rows * h8;
+  bool inf = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / h8;
     const int c = (int)(i - row * h8);
     const uint4 v = x[(int64_t)(perm[row] / K) * h8 + c];
-    out[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+    const uint4 o = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+    inf |= f16x2_has_inf(o.x) | f16x2_has_inf(o.y) | f16x2_has_inf(o.z) | f16x2_has_inf(o.w);
+    out[i] = o;
   }
+  if (inf) set_error(kErrF16Range);
 }
 
 // Router weight fp32 [n] -> three bf16 parts hi, mid, lo with w = hi + mid + lo

@@ -1,0 +1,164 @@
+"""GPU parity at the edges of the number formats, on both expert paths.
+
+Weights: E8M0 exponents spread far beyond the workloads' [118, 124]: uniform
+over [96, 140] (rows mixing groups 44 octaves apart) and over [0, 230] (nearly
+every representable scale; 230 keeps every fp32 intermediate of a V4-shape
+layer finite).  Activations: outlier channels a thousand times the rest,
+all-zero 32-value groups, groups near 2^-20, and a few values beyond the f16
+range (|x| > 65504).  Each case runs moe_expert_gemm at a decode size (the
+block-scaled path) and at a size above 8 pairs per expert, compares sampled
+pairs against the fp64 oracle at the layer tolerance, and checks the device
+status the call leaves.  A whole layer with every activation edge at once is
+checked at decode size (routing bit-exact through the gap-redrawn inputs).
+"""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from tests.cases import DeviceCase, make_case, oracle_pairs, rel_errors
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - CPU container
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import mxfp4_routed_expert_sqrt_b200 as m  # noqa: E402
+
+MAX_TOL, MEAN_TOL = 1e-2, 2e-3
+DEV = torch.device("cuda:0")
+V4 = gen.V4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    import __graft_entry__
+    __graft_entry__.build()
+    assert m.moe_device_error() == 0
+    yield
+    assert m.moe_device_error() == 0
+
+
+def _edit(fn):
+    """Wraps an fp32 edit of one activation row as an edit of its bf16 bits."""
+    def edit(t, row_bits):
+        v = gen.bf16_bits_to_f32(row_bits).astype(np.float32)
+        return gen.f32_to_bf16_bits(fn(t, v))
+    return edit
+
+
+OUTLIER_CH = np.array([5, 77, 1000, 2047, 2048, 3001, 4000, 4095])
+
+
+def outliers(t, v):
+    v[OUTLIER_CH] *= 1000.0
+    return v
+
+
+def zero_groups(t, v):
+    v.reshape(-1, 32)[t % 4::4] = 0.0
+    return v
+
+
+def tiny_groups(t, v):
+    v.reshape(-1, 32)[(t + 1) % 3::3] *= 2.0 ** -20
+    return v
+
+
+def beyond_f16(t, v):
+    v[[t % 4096, (7 * t + 3) % 4096]] = (1.0e5, -2.5e5)
+    return v
+
+
+def all_edges(t, v):
+    return beyond_f16(t, tiny_groups(t, zero_groups(t, outliers(t, v))))
+
+
+def _expert_gemm(dc, T):
+    c = dc.case
+    d = c.dims
+    H, I, E, K = d.hidden, d.inter, d.n_experts, d.top_k
+    idx = torch.empty(T * K, dtype=torch.int32, device=DEV)
+    w = torch.empty(T * K, dtype=torch.float32, device=DEV)
+    nb = m.moe_route_workspace_size(d, T)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=DEV)
+    m.moe_route(d, dc.x, T, dc.router, None, None, None, 0, idx, w, ws, nb)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * K, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * K, dtype=torch.int32, device=DEV)
+    m.moe_permute(idx, T, K, E, off, perm, inv)
+    y = torch.empty(T * K * H, dtype=torch.float32, device=DEV)
+    nb = m.moe_expert_gemm_workspace_size(d, T)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=DEV)
+    m.moe_expert_gemm(d, dc.x, T, m.proj(dc.gate, I, H), m.proj(dc.up, I, H), m.proj(dc.down, H, I), off, perm,
+                      y, ws, nb)
+    torch.cuda.synchronize()
+    return (idx.view(T, K).cpu().numpy(), perm.cpu().numpy(), y.view(T * K, H).cpu().numpy())
+
+
+def _dequant_path(T):
+    """The library's path choice (include/moe.h): more than 8 pairs per expert
+    on average runs the dequantising kernel."""
+    return -(-T * V4.top_k // V4.n_experts) > 8
+
+
+# (name, e_range, x_edit)
+EDGE_CASES = [
+    ("w_e96_140", (96, 140), None),
+    ("w_e0_230", (0, 230), None),
+    ("x_outliers", None, outliers),
+    ("x_zero_groups", None, zero_groups),
+    ("x_tiny_groups", None, tiny_groups),
+    ("x_beyond_f16", None, beyond_f16),
+    ("x_all_edges_w_e96_140", (96, 140), all_edges),
+]
+
+
+@pytest.mark.parametrize("T", [8, 400], ids=["decode_T8", "T400"])
+@pytest.mark.parametrize("name,e_range,x_edit", EDGE_CASES, ids=[c[0] for c in EDGE_CASES])
+def test_expert_gemm_edges(name, e_range, x_edit, T):
+    c = make_case(V4, T, seed=7, with_shared=False, e_range=e_range,
+                  x_edit=None if x_edit is None else _edit(x_edit))
+    dc = DeviceCase(c, DEV)
+    idx, perm, y = _expert_gemm(dc, T)
+    status = m.moe_device_error()
+    K = V4.top_k
+    rng = np.random.default_rng(T)
+    positions = np.unique(rng.choice(T * K, size=min(48, T * K), replace=False))
+    dequant = _dequant_path(T)
+    wide = e_range is not None and e_range[1] - e_range[0] > 36
+    big_x = x_edit in (beyond_f16, all_edges)
+    if dequant and big_x:
+        # activations beyond f16 cannot enter the f16 MMAs: refused with a status
+        assert status == m.DEVICE_ERR_F16_RANGE, hex(status)
+        return
+    if dequant and wide:
+        # groups more than 36 octaves below their row's largest are flushed, flagged
+        assert status == m.DEVICE_ERR_SPAN_FLUSH, hex(status)
+    else:
+        assert status == 0, hex(status)
+    got = y[positions]
+    assert np.isfinite(got).all()
+    want = oracle_pairs(c, idx, perm, positions)
+    mx, mean = rel_errors(got, want)
+    assert mx <= MAX_TOL and mean <= MEAN_TOL, f"{name} T={T}: max {mx:.2e} mean {mean:.2e}"
+
+
+def test_layer_with_every_activation_edge():
+    T = 32
+    c = make_case(V4, T, seed=9, e_range=(96, 140), x_edit=_edit(all_edges))
+    assert c.min_gap > 1e-4
+    dc = DeviceCase(c, DEV)
+    layer = m.MoeLayer(V4, T, DEV)
+    out = torch.empty(T * V4.hidden, dtype=torch.float32, device=DEV)
+    layer.forward(dc.weights, dc.x, T, out)
+    torch.cuda.synchronize()
+    assert m.moe_device_error() == 0
+    got = out.view(T, V4.hidden).cpu().numpy()
+    sel = np.arange(0, T, 4)
+    ridx, _, _, _ = oracle.route(c.x[sel], c.router, None, V4.top_k, V4.route_scale)
+    gb, ub, db = c.blobs_for(np.unique(ridx))
+    want, _, _ = oracle.moe_layer(V4, c.x, sel, c.router, None, gb, ub, db, shared=c.shared)
+    mx, mean = rel_errors(got[sel], want)
+    assert mx <= MAX_TOL and mean <= MEAN_TOL, f"max {mx:.2e} mean {mean:.2e}"

@@ -10,7 +10,7 @@ import pytest
 
 import gen
 import oracle
-from tests.cases import DeviceCase, make_case, rel_errors
+from tests.cases import DeviceCase, make_case, oracle_pairs, rel_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -192,12 +192,16 @@ EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64, None), ("tiny_T37", gen.TINY, 37, 7
                 # the two sides of the path switch: 8 pairs per expert on average
                 # (the largest block-scaled call), then 9 (the smallest dequantising one)
                 ("v4_T341_block_scaled_max", gen.V4, 341, 24, None),
-                ("v4_T342_dequant_min", gen.V4, 342, 24, None)]
+                ("v4_T342_dequant_min", gen.V4, 342, 24, None),
+                # the prefill size: 256 pairs spread over the call plus every pair of
+                # the four most loaded experts (each of their chunk positions)
+                ("v4_T4096_prefill", gen.V4, 4096, 256, "chunks")]
 
 
 @pytest.mark.parametrize("name,dims,T,nsample,bias", EXPERT_CASES, ids=[c[0] for c in EXPERT_CASES])
 def test_expert_gemm_parity(name, dims, T, nsample, bias):
     c = make_case(dims, T, with_shared=False, bias=_zipf_bias() if bias == "zipf" else None)
+    assert c.min_gap > 1e-4
     dc = DeviceCase(c, DEV)
     idx, perm, y = _expert_gemm(dc, T)
     K = dims.top_k
@@ -210,18 +214,19 @@ def test_expert_gemm_parity(name, dims, T, nsample, bias):
         start = int(counts[:hot].sum())
         edges = [j for b in range(32, int(counts[hot]), 32) for j in (b - 1, b)] + [0, int(counts[hot]) - 1]
         positions = np.concatenate([positions, start + np.array(edges)])
+    if bias == "chunks":
+        # every position of a chunk: all pairs of the experts that hold the
+        # sampled positions' neighbours at chunk starts, middles and ends
+        counts = np.bincount(idx.reshape(-1), minlength=dims.n_experts)
+        starts = np.concatenate([[0], np.cumsum(counts)])
+        extra = []
+        for e in np.argsort(-counts)[:4]:
+            extra.extend(range(int(starts[e]), int(starts[e + 1])))
+        positions = np.concatenate([positions, np.array(extra, np.int64)])
     positions = np.unique(positions)
-    xs_all = (c.x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    got, want = [], []
-    for pos in positions:
-        p = perm[pos]
-        t, k = divmod(int(p), K)
-        e = int(idx[t, k])
-        ref = oracle.expert_ffn(c.blob("gate", e), c.blob("up", e), c.blob("down", e), dims.hidden, dims.inter,
-                                dims.swiglu_limit, xs_all[t:t + 1])
-        got.append(y[pos])
-        want.append(ref[0])
-    mx, mean = rel_errors(np.array(got), np.array(want))
+    got = y[positions]
+    want = oracle_pairs(c, idx, perm, positions)
+    mx, mean = rel_errors(got, want)
     assert mx <= MAX_TOL and mean <= MEAN_TOL, f"{name}: max {mx:.2e} mean {mean:.2e}"
 
 
@@ -280,7 +285,7 @@ LAYER_CASES = [("tiny_T8", gen.TINY, 8, None, False, 8), ("tiny_T1", gen.TINY, 1
                ("v4_zipf_T32_layer0", gen.V4, 32, "zipf", False, 8),
                ("v4_decode_T1", gen.V4, 1, None, False, 1), ("v4_decode_T8", gen.V4, 8, None, False, 8),
                ("v4_decode_T32", gen.V4, 32, None, False, 8), ("v4_decode_T64", gen.V4, 64, None, False, 8),
-               ("v4_hash_T2048", gen.V4, 2048, None, True, 6), ("v4_prefill_T4096", gen.V4, 4096, None, False, 6),
+               ("v4_hash_T2048", gen.V4, 2048, None, True, 6), ("v4_prefill_T4096", gen.V4, 4096, None, False, 48),
                # degenerate routing: every table row names the same 6 experts, so all
                # 1,800 pairs land on them (ten 32-pair chunks each) and 250 experts are empty
                ("v4_hash_all_same_T300", gen.V4, 300, None, "same", 6)]

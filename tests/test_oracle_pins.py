@@ -275,27 +275,40 @@ def _tiny_layer_blobs(seed=0, layer=0):
     return gates, ups, downs
 
 
-@pytest.mark.parametrize("hashed", [False, True])
-def test_tiny_layer_equals_dense_bruteforce(oracle_lib, hashed):
-    """Tiny config: every expert evaluated densely and masked by the routing."""
+@pytest.mark.parametrize("mode", ["learned", "learned_bias", "hashed"])
+def test_tiny_layer_equals_dense_bruteforce(oracle_lib, mode):
+    """Tiny config: every expert evaluated densely and masked by the routing.
+    With a selection bias strong enough to change which experts win, the
+    layer must route through it (a layer that dropped the bias on its way to
+    the router would pick different experts and fail)."""
     d = gen.TINY
     T = 8
     x = gen.x_rows(0, 0, T, d.hidden)
     wr = gen.router_weight(0, 0, d.n_experts, d.hidden)
     gates, ups, downs = _tiny_layer_blobs()
     shared = gen.shared_weights(0, 0, d.hidden, d.inter)
-    tok = table = None
-    if hashed:
+    tok = table = bias = None
+    if mode == "hashed":
         table = gen.hash_table(0, 64, d.n_experts, d.top_k)
         tok = gen.token_ids(0, 0, T, 64)
-    out, idx, w = oracle_lib.moe_layer(d, x, np.arange(T), wr, None, gates, ups, downs,
+    if mode == "learned_bias":
+        bias = gen.zipf_bias(0, d.n_experts, 0.6)
+    out, idx, w = oracle_lib.moe_layer(d, x, np.arange(T), wr, bias, gates, ups, downs,
                                        shared=shared, tok=tok, table=table, nthreads=4)
-    want, mask = indep.dense_layer(d, x, wr, None, gates, ups, downs, shared=shared, tok=tok, table=table)
+    want, mask = indep.dense_layer(d, x, wr, bias, gates, ups, downs, shared=shared, tok=tok, table=table)
     assert np.allclose(out, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
     for t in range(T):
         assert np.allclose(mask[t, idx[t]], w[t], rtol=1e-13)
+    if mode == "learned_bias":
+        # the bias changes the selection of some tokens, and the unbiased
+        # layer differs from the biased one there
+        nob, idx0, _ = oracle_lib.moe_layer(d, x, np.arange(T), wr, None, gates, ups, downs,
+                                            shared=shared, nthreads=4)
+        changed = [t for t in range(T) if set(idx0[t]) != set(idx[t])]
+        assert changed, "the bias must change at least one token's experts"
+        assert not np.allclose(nob[changed], out[changed])
     # a subset of tokens gives exactly those rows
-    sub, _, _ = oracle_lib.moe_layer(d, x, np.array([5, 2]), wr, None, gates, ups, downs,
+    sub, _, _ = oracle_lib.moe_layer(d, x, np.array([5, 2]), wr, bias, gates, ups, downs,
                                      shared=shared, tok=tok, table=table, nthreads=2)
     assert np.array_equal(sub, out[[5, 2]])
 

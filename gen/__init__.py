@@ -15,7 +15,8 @@ oracle regenerates any single expert on the host.
 Input recipe (the shapes and distributions of the V4-Flash workloads):
   * routed expert weights: E2M1 codes uniform over the 16 codes (each byte of
     the nibble plane uniform over 256), E8M0 exponents uniform over [lo, hi]
-    (default [118, 124]);
+    (default [118, 124]), or, for edge cases, a uniform base per weight row
+    plus a small uniform offset per group;
   * activations X ~ N(0, 1) rounded to bf16, one independent sub-stream per
     (token row, attempt) so a row can be redrawn;
   * router weight ~ N(0, 1/H) in fp32; shared-expert weights ~ N(0, 1/fan_in)
@@ -44,6 +45,7 @@ T_SHARED_GATE, T_SHARED_UP, T_SHARED_DOWN = 4, 5, 6
 T_CODES = {"gate": 7, "up": 9, "down": 11}
 T_SCALES = {"gate": 8, "up": 10, "down": 12}
 T_HASH_TABLE, T_TOKEN_IDS, T_CALIB_X = 13, 14, 15
+T_ROW_BASE = {"gate": 16, "up": 17, "down": 18}
 
 E8M0_LO, E8M0_HI = 118, 124
 
@@ -129,9 +131,19 @@ def blob_layout(rows: int, cols: int):
     return nib, sc, nib + sc
 
 
+def _below(r: np.ndarray, n: int) -> np.ndarray:
+    """Integers in [0, n) from the high 32 bits of uint64 draws (multiply-shift)."""
+    return ((r >> np.uint64(32)) * np.uint64(n)) >> np.uint64(32)
+
+
 def mxfp4_expert_host(seed: int, layer: int, proj: str, x: int, rows: int, cols: int,
-                      e_lo: int = E8M0_LO, e_hi: int = E8M0_HI) -> np.ndarray:
-    """Bytes of expert ``x`` of one projection, identical to the device fill."""
+                      e_lo: int = E8M0_LO, e_hi: int = E8M0_HI, row_span: int = -1) -> np.ndarray:
+    """Bytes of expert ``x`` of one projection, identical to the device fill.
+
+    row_span < 0: every E8M0 byte uniform over [e_lo, e_hi].  row_span >= 0:
+    each weight row draws a base uniform over [e_lo, e_hi - row_span] (from
+    its own stream, counter = global row x * rows + r) and its bytes are the
+    base plus a uniform offset in [0, row_span]."""
     nib, sc, total = blob_layout(rows, cols)
     assert nib % 8 == 0
     kc = derive(seed, layer, T_CODES[proj])
@@ -140,8 +152,14 @@ def mxfp4_expert_host(seed: int, layer: int, proj: str, x: int, rows: int, cols:
     w0 = x * (nib // 8)
     out[:nib] = u64(kc, np.arange(w0, w0 + nib // 8, dtype=np.uint64)).view(np.uint8)
     r = u64(ks, np.arange(x * sc, (x + 1) * sc, dtype=np.uint64))
-    span = np.uint64(e_hi - e_lo + 1)
-    out[nib:] = (np.uint64(e_lo) + (((r >> np.uint64(32)) * span) >> np.uint64(32))).astype(np.uint8)
+    if row_span < 0:
+        out[nib:] = (np.uint64(e_lo) + _below(r, e_hi - e_lo + 1)).astype(np.uint8)
+    else:
+        kr = derive(seed, layer, T_ROW_BASE[proj])
+        per_row = cols // 32
+        grow = np.uint64(x * rows) + np.arange(sc, dtype=np.uint64) // np.uint64(per_row)
+        base = np.uint64(e_lo) + _below(u64(kr, grow), e_hi - row_span - e_lo + 1)
+        out[nib:] = (base + _below(r, row_span + 1)).astype(np.uint8)
     return out
 
 
@@ -158,19 +176,22 @@ def _load_device_lib():
         lib.moegen_fill_mxfp4.restype = ctypes.c_int
         lib.moegen_fill_mxfp4.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                           ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64,
-                                          ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+                                          ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_void_p]
         _lib = lib
     return _lib
 
 
 def mxfp4_fill_device(dst_ptr: int, stream_ptr: int, seed: int, layer: int, proj: str,
                       n_experts: int, rows: int, cols: int,
-                      e_lo: int = E8M0_LO, e_hi: int = E8M0_HI) -> None:
-    """Fill n_experts back-to-back blobs at device address dst_ptr on a stream."""
+                      e_lo: int = E8M0_LO, e_hi: int = E8M0_HI, row_span: int = -1) -> None:
+    """Fill n_experts back-to-back blobs at device address dst_ptr on a stream
+    (the same bytes as mxfp4_expert_host for every expert)."""
     lib = _load_device_lib()
     rc = lib.moegen_fill_mxfp4(ctypes.c_void_p(dst_ptr), n_experts, rows, cols,
                                derive(seed, layer, T_CODES[proj]),
-                               derive(seed, layer, T_SCALES[proj]), e_lo, e_hi,
+                               derive(seed, layer, T_SCALES[proj]),
+                               derive(seed, layer, T_ROW_BASE[proj]), e_lo, e_hi, row_span,
                                ctypes.c_void_p(stream_ptr))
     if rc != 0:
         raise RuntimeError(f"moegen_fill_mxfp4 failed with CUDA error {rc}")

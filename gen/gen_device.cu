@@ -33,30 +33,43 @@ __global__ void fill_codes(uint8_t* base, int64_t n_experts, int64_t nib_words,
   }
 }
 
-__global__ void fill_scales(uint8_t* base, int64_t n_experts, int64_t nib_bytes,
-                            int64_t sc_bytes, int64_t expert_bytes, uint64_t key,
-                            uint32_t lo, uint32_t span) {
+__device__ __forceinline__ uint32_t below(uint64_t r, uint32_t n) { return (uint32_t)(((r >> 32) * n) >> 32); }
+
+// row_span < 0: byte = lo + below(draw, span).  row_span >= 0: byte = base of
+// the weight row (lo + below(row draw, span - row_span), row draw = output
+// x * rows + r of the row stream) + below(draw, row_span + 1).
+__global__ void fill_scales(uint8_t* base, int64_t n_experts, int64_t rows, int64_t per_row, int64_t nib_bytes,
+                            int64_t sc_bytes, int64_t expert_bytes, uint64_t key, uint64_t key_rows,
+                            uint32_t lo, uint32_t span, int row_span) {
   const int64_t total = n_experts * sc_bytes;
   for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < total;
        j += (int64_t)gridDim.x * blockDim.x) {
     const int64_t x = j / sc_bytes, i = j % sc_bytes;
     const uint64_t r = mix64(key + (uint64_t)(j + 1) * kGolden);
-    base[x * expert_bytes + nib_bytes + i] = (uint8_t)(lo + (((r >> 32) * span) >> 32));
+    uint32_t v;
+    if (row_span < 0) {
+      v = lo + below(r, span);
+    } else {
+      const uint64_t grow = (uint64_t)(x * rows + i / per_row);
+      const uint64_t rb = mix64(key_rows + (grow + 1) * kGolden);
+      v = lo + below(rb, span - (uint32_t)row_span) + below(r, (uint32_t)row_span + 1);
+    }
+    base[x * expert_bytes + nib_bytes + i] = (uint8_t)v;
   }
 }
 
 }  // namespace
 
 extern "C" int moegen_fill_mxfp4(uint8_t* base, int64_t n_experts, int64_t rows, int64_t cols,
-                                 uint64_t key_codes, uint64_t key_scales, int e_lo, int e_hi,
-                                 cudaStream_t stream) {
+                                 uint64_t key_codes, uint64_t key_scales, uint64_t key_rows, int e_lo,
+                                 int e_hi, int row_span, cudaStream_t stream) {
   if (!base || n_experts <= 0 || rows <= 0 || cols <= 0 || cols % 32 != 0 ||
-      ((uintptr_t)base & 31) || e_lo < 0 || e_hi > 254 || e_lo > e_hi)
+      ((uintptr_t)base & 31) || e_lo < 0 || e_hi > 254 || e_lo > e_hi || row_span > e_hi - e_lo)
     return (int)cudaErrorInvalidValue;
   const int64_t nib = rows * cols / 2, sc = rows * cols / 32, eb = nib + sc;
   if (nib % 8 != 0) return (int)cudaErrorInvalidValue;
   fill_codes<<<148 * 8, 256, 0, stream>>>(base, n_experts, nib / 8, eb, key_codes);
-  fill_scales<<<148 * 4, 256, 0, stream>>>(base, n_experts, nib, sc, eb, key_scales,
-                                           (uint32_t)e_lo, (uint32_t)(e_hi - e_lo + 1));
+  fill_scales<<<148 * 4, 256, 0, stream>>>(base, n_experts, rows, cols / 32, nib, sc, eb, key_scales, key_rows,
+                                           (uint32_t)e_lo, (uint32_t)(e_hi - e_lo + 1), row_span);
   return (int)cudaGetLastError();
 }

@@ -226,10 +226,24 @@ class LayerWeights:
     hash_table: object = None   # int32 [vocab, K] for hash-routed layers
 
 
+def _torch_stream(s):
+    """A torch stream object for `s` (None: the current stream; an int: a raw
+    cudaStream_t)."""
+    import torch
+    if s is None:
+        return torch.cuda.current_stream()
+    if isinstance(s, int):
+        return torch.cuda.ExternalStream(s)
+    return s
+
+
 class MoeLayer:
-    """Runs route -> permute -> experts -> shared -> combine for up to max_T
-    tokens on one stream.  Workspaces and intermediates are allocated once
-    (torch) for max_T; a forward allocates nothing."""
+    """Runs route -> permute -> experts -> combine for up to max_T tokens on
+    the caller's stream, with the shared expert (which needs only x) on a
+    side stream forked at the start of the layer and joined before the
+    combine, so it overlaps routing and grouping.  Workspaces and
+    intermediates are allocated once (torch) for max_T; a forward allocates
+    nothing and can be captured in a CUDA graph."""
 
     def __init__(self, dims, max_T: int, device=None):
         import torch
@@ -253,6 +267,7 @@ class MoeLayer:
         self.ws_perm = torch.empty(max(self.ws_perm_bytes, 256), dtype=torch.uint8, device=dev)
         self.ws_exp = torch.empty(max(self.ws_exp_bytes, 256), dtype=torch.uint8, device=dev)
         self.ws_sh = torch.empty(max(self.ws_sh_bytes, 256), dtype=torch.uint8, device=dev)
+        self.side = torch.cuda.Stream(device=dev)  # the shared expert's stream
 
     def forward(self, w: LayerWeights, x, T: int, out_f32, token_ids=None, out_bf16=None, stream=None,
                 expert_events=None):
@@ -264,25 +279,35 @@ class MoeLayer:
         H, I, E, K = d.hidden, d.inter, d.n_experts, d.top_k
         if T > self.max_T:
             raise ValueError(f"T={T} exceeds max_T={self.max_T}")
+        import torch
         hashed = w.hash_table is not None
         vocab = w.hash_table.shape[0] if hashed else 0
-        moe_route(d, x, T, w.router_w, None if hashed else w.bias, token_ids if hashed else None,
-                  w.hash_table if hashed else None, vocab, self.topk_idx, self.topk_w, self.ws_route,
-                  self.ws_route_bytes, stream)
-        moe_permute(self.topk_idx, T, K, E, self.offsets, self.perm, self.inv, self.ws_perm,
-                    self.ws_perm_bytes, stream)
+        main = _torch_stream(stream)
         has_shared = w.shared_gate is not None
         if has_shared:
+            # fork: the shared expert runs beside routing and grouping
+            fork = torch.cuda.Event()
+            fork.record(main)
+            self.side.wait_event(fork)
             shared_expert(d, x, T, w.shared_gate, w.shared_up, w.shared_down, self.shared_out, self.ws_sh,
-                          self.ws_sh_bytes, stream)
+                          self.ws_sh_bytes, self.side)
+            join = torch.cuda.Event()
+            join.record(self.side)
+        moe_route(d, x, T, w.router_w, None if hashed else w.bias, token_ids if hashed else None,
+                  w.hash_table if hashed else None, vocab, self.topk_idx, self.topk_w, self.ws_route,
+                  self.ws_route_bytes, main)
+        moe_permute(self.topk_idx, T, K, E, self.offsets, self.perm, self.inv, self.ws_perm,
+                    self.ws_perm_bytes, main)
         if expert_events is not None:
-            expert_events[0].record()
+            expert_events[0].record(main)
         moe_expert_gemm(d, x, T, proj(w.gate, I, H), proj(w.up, I, H), proj(w.down, H, I), self.offsets,
-                        self.perm, self.y_perm, self.ws_exp, self.ws_exp_bytes, stream)
+                        self.perm, self.y_perm, self.ws_exp, self.ws_exp_bytes, main)
         if expert_events is not None:
-            expert_events[1].record()
+            expert_events[1].record(main)
+        if has_shared:
+            main.wait_event(join)  # join
         moe_combine(d, T, self.y_perm, self.inv, self.topk_w, self.shared_out if has_shared else None,
-                    out_f32, out_bf16, stream)
+                    out_f32, out_bf16, main)
         return out_f32
 
     def graphed(self, w: LayerWeights, T: int, host_x, host_out, token_ids=None, stream=None):

@@ -17,6 +17,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y_perm, const int32_t* __restrict__ inv,
     const float* __restrict__ w, const float* __restrict__ shared, float* __restrict__ out,
     __nv_bfloat16* __restrict__ out_bf16, int K, int H) {
+  griddep_wait();
+  griddep_launch();
   const int t = blockIdx.y;
   const int c4 = blockIdx.x * kCombineThreads + threadIdx.x;
   if (c4 * 4 >= H) return;

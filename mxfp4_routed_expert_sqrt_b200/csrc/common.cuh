@@ -24,6 +24,16 @@ enum : int32_t {
 
 __device__ int32_t g_error;
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may begin while its predecessor in the stream is finishing;
+// griddep_wait() returns once every prerequisite grid has completed and its
+// memory is visible, so each kernel calls it before its first global read or
+// write.  griddep_launch() lets the stream's next kernel begin launching (its
+// CTAs then wait in their own griddep_wait()).  Without the launch attribute
+// both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_error(int32_t code) { atomicCAS(&g_error, 0, code); }
 
 // Upper bound on the time a kernel waits for one mbarrier phase before it

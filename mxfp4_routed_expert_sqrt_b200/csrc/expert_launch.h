@@ -22,17 +22,41 @@ inline int expert_chunk(int T, int K, int E) {
   return avg <= 8 ? 32 : avg <= 24 ? 64 : kTcNMax;
 }
 
+// Mean pairs per expert up to which moe_expert_gemm takes the block-scaled
+// kernel; above it, the kernel that dequantises to f16.
+constexpr int kBlockScaledMaxAvg = 8;
+
 // Path choice from the host-known T: with few pairs per expert (32-pair
 // chunks, decode) the weights stream through the block-scaled kernel; with
 // many, the kernel that dequantises to f16 keeps 128-token units, double the
 // epilogue warps and one read of each expert's weights.
-inline bool use_block_scaled(int T, int K, int E) { return expert_chunk(T, K, E) <= 32; }
+inline bool use_block_scaled(int T, int K, int E) {
+  return ((int64_t)T * K + E - 1) / E <= kBlockScaledMaxAvg;
+}
 
 // E4M3 terms of the activations (exact for bf16) and of h between the GEMMs
-// on the block-scaled path: three terms of h for 32-pair chunks (N = 96).
+// on the block-scaled path (three terms of h: about 12 significant bits).
 constexpr int kXTerms = 2;
 constexpr int kHTerms = 3;
-constexpr int kMxChunk = 32;
+
+// Token layout of the block-scaled kernel by mean pairs per expert: up to 8,
+// the terms stacked along N in 32-pair chunks (N 64 and 96 cost what N 16
+// does) with one accumulator set; up to 24, the terms summed into one
+// accumulator in 64-pair chunks with two accumulator sets (a unit's epilogue
+// overlaps the next unit's MMAs); above, 128-pair chunks (N 128, the MMA's
+// efficient width; one set fits), so an expert's weights are read once per
+// 128 of its pairs.
+struct MxLayout {
+  int chunk, term_acc, max_bufs;
+};
+constexpr int kMxDecodeBufs = 1;  // accumulator sets of the stacked (decode) layout
+constexpr int kMxPrefetchKt = 0;  // K-tiles of weights the loader prefetches into L2 ahead
+inline MxLayout mx_layout(int T, int K, int E) {
+  const int64_t avg = ((int64_t)T * K + E - 1) / E;
+  if (avg <= 8) return {32, 0, kMxDecodeBufs};
+  if (avg <= 24) return {64, 1, 2};
+  return {128, 1, 2};
+}
 
 // The block-scaled path's workspace: E4M3 terms and E8M0 scales of the pairs'
 // activations in expert order, then of h: [2][pairs][hidden],
@@ -77,7 +101,11 @@ inline bool mx_launch_args(const moe_dims& dims, int T, const moe_mxfp4_proj& ga
   g.pairs = (int)L.pairs;
   g.parts = kXTerms;
   g.b_scale = L.xs;
-  g.n_chunk = kMxChunk;
+  const MxLayout lay = mx_layout(T, dims.top_k, dims.n_experts);
+  g.n_chunk = lay.chunk;
+  g.term_acc = lay.term_acc;
+  g.max_bufs = lay.max_bufs;
+  g.prefetch = kMxPrefetchKt;
   g.out = L.hq;
   g.out_scale = L.hs;
   g.out_parts = kHTerms;

@@ -50,6 +50,33 @@ moe_status launch_status() {
   return MOE_OK;
 }
 
+// Kernels are launched with programmatic stream serialization: each one may
+// begin (its prologue: barriers, TMEM, descriptor fetches) while its
+// predecessor in the stream finishes, and waits in griddep_wait() before its
+// first global access, so stream order holds for every byte.
+constexpr bool kUsePdl = true;
+
+template <typename... KArgs, typename... Args>
+moe_status launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                    const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "libmoe: launch failed: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -134,8 +161,8 @@ moe_status launch_tc_epi(const CUtensorMap& bmap, TcArgs a, cudaStream_t s) {
   } else {
     w1 = w0;
   }
-  tc_expert_kernel<MODE, AF, EPI><<<sm_count(), tc_threads(EPI), a.smem_bytes, s>>>(bmap, w0, w1, a);
-  return launch_status();
+  return launch_k(tc_expert_kernel<MODE, AF, EPI>, dim3(sm_count()), dim3(tc_threads(EPI)), a.smem_bytes, s, bmap, w0,
+                  w1, a);
 }
 
 // 128-token chunks get 8 epilogue warps, smaller ones 4.
@@ -170,20 +197,57 @@ bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// E8M0 plane of an MXFP4 weight array: {row bytes (cols / 32), rows, experts}
+// with boxes of one scale stage's bytes (4 G) of 128 rows, no swizzle.
+bool make_mx_scale_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr || base == nullptr) return false;
+  const int64_t plane = (int64_t)a.rows * (a.cols / 2);
+  cuuint64_t dims[3] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.rows, (cuuint64_t)a.E};
+  cuuint64_t strides[2] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.expert_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(4 * a.g), 128, 1}, estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base + plane), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E8M0 scales of the token terms [parts * pairs][cols / 32] with boxes of one
+// scale stage's bytes of 16 rows, no swizzle.
+bool make_token_scale_map(CUtensorMap* map, const MxArgs& a) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr || a.b_scale == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.parts * a.pairs};
+  cuuint64_t strides[1] = {(cuuint64_t)a.cols / 32};
+  cuuint32_t box[2] = {(cuuint32_t)(4 * a.g), (cuuint32_t)kTcBoxRows}, estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.b_scale), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // One block-scaled expert launch (planned by mx_plan), one CTA per SM.
 template <int MODE, int G>
 moe_status launch_mx_g(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
   static std::atomic<uint64_t> configured{0};
   if (!smem_limit_once(configured, mx_expert_kernel<MODE, G>, kTcSmemMax)) return MOE_ERR_CUDA;
-  CUtensorMap w0, w1;
+  CUtensorMap w0, w1, s0, s1, ts;
   if (!make_mx_weight_map(&w0, a.w0, a)) return MOE_ERR_CUDA;
   if (MODE == 0) {
     if (!make_mx_weight_map(&w1, a.w1, a)) return MOE_ERR_CUDA;
   } else {
     w1 = w0;
   }
-  mx_expert_kernel<MODE, G><<<sm_count(), kMxThreads, a.smem_bytes, s>>>(bmap, w0, w1, a);
-  return launch_status();
+  if (a.tma_scales) {
+    if (!make_mx_scale_map(&s0, a.w0, a) || !make_token_scale_map(&ts, a)) return MOE_ERR_CUDA;
+    if (MODE == 0) {
+      if (!make_mx_scale_map(&s1, a.w1, a)) return MOE_ERR_CUDA;
+    } else {
+      s1 = s0;
+    }
+  } else {  // unused: the scale writers load the E8M0 rows themselves
+    s0 = s1 = ts = w0;
+  }
+  return launch_k(mx_expert_kernel<MODE, G>, dim3(sm_count()), dim3(kMxThreads), a.smem_bytes, s, bmap, w0, w1, s0,
+                  s1, ts, a);
 }
 
 template <int MODE>
@@ -347,8 +411,8 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
     // logits = x . (hi + mid + lo) on the tensor cores: every product exact, fp32 sums
     __nv_bfloat16* split = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) +
                                                             round_up((size_t)T * E * sizeof(float), 256));
-    split3_bf16_kernel<<<2 * sm_count(), 256, 0, s>>>(router_w, split, E, H);
-    if ((st = launch_status()) != MOE_OK) return st;
+    if ((st = launch_k(split3_bf16_kernel, dim3(2 * sm_count()), dim3(256), 0, s, router_w, split, E, H)) != MOE_OK)
+      return st;
     CUtensorMap xmap;
     if (!make_row_map(&xmap, x, T, H)) return MOE_ERR_CUDA;
     TcArgs a{};
@@ -363,14 +427,13 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
     if ((st = launch_tc<1, kABf16>(xmap, a, s)) != MOE_OK) return st;
   } else {
     dim3 g1((E + kLogitExperts - 1) / kLogitExperts, (T + kLogitTokBlock - 1) / kLogitTokBlock);
-    route_logits_kernel<<<g1, kLogitThreads, kLogitExperts * H * sizeof(float), s>>>(
-        static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits);
-    if ((st = launch_status()) != MOE_OK) return st;
+    if ((st = launch_k(route_logits_kernel, g1, dim3(kLogitThreads), kLogitExperts * H * sizeof(float), s,
+                       static_cast<const __nv_bfloat16*>(x), T, H, router_w, E, logits)) != MOE_OK)
+      return st;
   }
-  route_select_kernel<<<(T + 3) / 4, 128, 4 * E * sizeof(float), s>>>(
-      logits, T, E, dims->top_k, dims->route_scale, hashed ? nullptr : bias, token_ids, hash_table,
-      vocab, topk_idx, topk_w);
-  return launch_status();
+  return launch_k(route_select_kernel, dim3((T + 3) / 4), dim3(128), 4 * E * sizeof(float), s,
+                  static_cast<const float*>(logits), T, E, dims->top_k, dims->route_scale,
+                  hashed ? nullptr : bias, token_ids, hash_table, vocab, topk_idx, topk_w);
 }
 
 moe_status moe_route_noalloc(const moe_dims* dims, const void* x, int32_t T, const float* router_w,
@@ -414,8 +477,7 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
   const int smem = 32 * E * (int)sizeof(int32_t);
   static std::atomic<uint64_t> configured{0};
   if (!smem_limit_once(configured, permute_kernel, 32 * 1024 * 4)) return MOE_ERR_CUDA;
-  permute_kernel<<<1, kPermuteThreads, smem, s>>>(topk_idx, T * K, E, offsets, perm, inv);
-  return launch_status();
+  return launch_k(permute_kernel, dim3(1), dim3(kPermuteThreads), smem, s, topk_idx, T * K, E, offsets, perm, inv);
 }
 
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
@@ -434,9 +496,9 @@ moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t
   const int H = dims->hidden, I = dims->inter;
   // the activations of every pair, in expert order, as E4M3 terms
   const int64_t n8 = L.pairs * H / 8;
-  gather_split_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
-      static_cast<const uint4*>(x), perm, dims->top_k, H, L.pairs, kXTerms, L.xq, L.xs);
-  moe_status st = launch_status();
+  moe_status st = launch_k(gather_split_kernel, dim3((int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184)),
+                           dim3(256), 0, s, static_cast<const uint4*>(x), perm, dims->top_k, H, L.pairs, kXTerms,
+                           L.xq, L.xs);
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
   if (!make_term_map(&xmap, L.xq, kXTerms * L.pairs, H) || !make_term_map(&hmap, L.hq, kHTerms * L.pairs, I))
@@ -455,9 +517,9 @@ moe_status expert_gemm_dequant(const moe_dims* dims, const void* x, int32_t T, c
   // the activations of every pair, in expert order and f16 (the token operand
   // of the gate/up GEMM is then read with plain TMA boxes)
   const int64_t n8 = L.pairs * H / 8;
-  gather_f16_kernel<<<(int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184), 256, 0, s>>>(
-      static_cast<const uint4*>(x), perm, dims->top_k, H / 8, L.pairs, reinterpret_cast<uint4*>(L.x16));
-  moe_status st = launch_status();
+  moe_status st = launch_k(gather_f16_kernel, dim3((int)((n8 + 255) / 256 < 4 * 1184 ? (n8 + 255) / 256 : 4 * 1184)),
+                           dim3(256), 0, s, static_cast<const uint4*>(x), perm, dims->top_k, H / 8, L.pairs,
+                           reinterpret_cast<uint4*>(L.x16));
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
   if (!make_row_map(&xmap, L.x16, L.pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -550,8 +612,7 @@ moe_status shared_expert(const moe_dims* dims, const void* x, int32_t T, const v
   g.T = T;
   g.out = h2;
   g.limit = dims->swiglu_limit;
-  shared_decode_kernel<0><<<I / 8, kShThreads, 0, s>>>(g);
-  if ((st = launch_status()) != MOE_OK) return st;
+  if ((st = launch_k(shared_decode_kernel<0>, dim3(I / 8), dim3(kShThreads), 0, s, g)) != MOE_OK) return st;
   ShArgs d = g;
   d.w0 = static_cast<const __nv_bfloat16*>(wd);
   d.w1 = nullptr;
@@ -560,8 +621,7 @@ moe_status shared_expert(const moe_dims* dims, const void* x, int32_t T, const v
   d.k_total = 2 * I;
   d.xin = h2;
   d.out = out;
-  shared_decode_kernel<1><<<H / 16, kShThreads, 0, s>>>(d);
-  return launch_status();
+  return launch_k(shared_decode_kernel<1>, dim3(H / 16), dim3(kShThreads), 0, s, d);
 }
 
 moe_status moe_combine(const moe_dims* dims, int32_t T, const float* y_perm, const int32_t* inv,
@@ -577,9 +637,8 @@ moe_status moe_combine(const moe_dims* dims, int32_t T, const float* y_perm, con
     return MOE_ERR_ALIGNMENT;
   const int H = dims->hidden;
   dim3 grid((H / 4 + kCombineThreads - 1) / kCombineThreads, T);
-  combine_kernel<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      y_perm, inv, topk_w, shared_out, out_f32, static_cast<__nv_bfloat16*>(out_bf16), dims->top_k, H);
-  return launch_status();
+  return launch_k(combine_kernel, grid, dim3(kCombineThreads), 0, static_cast<cudaStream_t>(stream), y_perm, inv,
+                  topk_w, shared_out, out_f32, static_cast<__nv_bfloat16*>(out_bf16), dims->top_k, H);
 }
 
 }  // extern "C"

@@ -14,12 +14,21 @@
 // The token operand is E4M3 with its own E8M0 group-32 scales.  Each
 // activation v is carried as a sum of `parts` E4M3 terms: term p encodes the
 // residual r_p = v - (terms 0 .. p-1) with the block scale 2^(floor(log2(max
-// |r_p| over the 32-value group)) - 7) and round-to-nearest-even.  Terms are
-// stacked along the MMA's N dimension (N = parts x tokens) and summed in fp32
-// by the epilogue.  Two terms carry a bf16 value exactly (8 significant bits
-// in two 4-bit terms) unless the residual of an element falls below the E4M3
-// normal range of its group; h between the GEMMs (fp32 in the epilogue) keeps
-// about 12 significant bits with three terms and about 8 with two.
+// |r_p| over the 32-value group)) - 7) and round-to-nearest-even.  Two terms
+// carry a bf16 value exactly (8 significant bits in two 4-bit terms) unless
+// the residual of an element falls below the E4M3 normal range of its group;
+// h between the GEMMs (fp32 in the epilogue) keeps about 12 significant bits
+// with three terms and about 8 with two.  The terms reach the tensor core in
+// one of two ways (args.term_acc):
+//   stacked  (0): along the MMA's N dimension (N = parts x tokens), summed in
+//                 fp32 by the epilogue -- free while N stays small (an MMA of
+//                 N <= 64 costs about what one of N 16 does), so decode
+//                 batches use it;
+//   summed   (1): one MMA per term into the same accumulator columns (the
+//                 product is linear in the token operand), N = tokens -- half
+//                 the accumulator columns per token, so chunks of 64-128
+//                 tokens (and two accumulator sets) fit in TMEM at larger
+//                 batches, where the MMA's cost grows with N anyway.
 //
 // Per unit = (expert e, token chunk of <= n_chunk grouped pairs, row tile):
 //   MODE 0 (gate/up): acc0 = Wg[128 rows] x^T, acc1 = Wu[128 rows] x^T over
@@ -44,12 +53,14 @@
 //              quadrant holding a full copy;
 //   warp 8     loader (one thread): TMA boxes of weights and token terms;
 //   warp 9     TMEM owner and MMA issuer (one thread).
-// TMEM (512 columns): acc0 [0, acc), acc1 [acc, 2 acc), then the scale ring.
-// A scale stage holds, for K-tile j of the stage, the weight scales at column
-// 8j + 4m + c (m = tile, c = row / 32) and the token scales at column
-// 8G + 4j + c (c = N index / 32); lane i of every quadrant holds rows (or N
-// indices) 32c + i; byte b of a column is k-block 4 kt + b, which the MMA
-// selects with the scale-factor id.
+// TMEM (512 columns): acc_bufs accumulator sets (set b: acc0 at 2 b acc,
+// acc1 at 2 b acc + acc), then the scale ring.  With two sets the epilogue of
+// one unit overlaps the MMAs of the next.  A scale stage holds, for K-tile j
+// of the stage, the weight scales at column 8j + 4m + c (m = tile, c = row /
+// 32) and the token scales at column 8G + tok_cols j + c: stacked, c = N
+// index / 32 (4 columns); summed, c = 4 p + token / 32 (4 columns per term).
+// Lane i of every quadrant holds rows (or N indices) 32c + i; byte b of a
+// column is k-block 4 kt + b, which the MMA selects with the scale-factor id.
 #pragma once
 
 #include <cuda.h>
@@ -66,8 +77,8 @@ constexpr int kMxTileTx = 8192;      // transaction bytes of that box (4 bits pe
 constexpr int kMxMaxStages = 8;
 constexpr int kMxMaxSfStages = 4;
 constexpr int kMxMaxParts = 3;
-constexpr int kMxNMax = 128;   // MMA N: terms x padded tokens
-constexpr int kMxSfPerKt = 12; // TMEM columns per K-tile in a scale stage (8 weight + 4 token)
+constexpr int kMxNMax = 128;   // MMA N: tokens (summed terms) or terms x padded tokens (stacked)
+constexpr int kMxMaxBufs = 2;  // accumulator sets
 
 struct MxArgs {
   const uint8_t* w0;     // MODE 0: gate; MODE 1: down
@@ -81,16 +92,25 @@ struct MxArgs {
   int parts;             // E4M3 terms of the token operand
   const uint8_t* b_scale;  // token E8M0 [parts][pairs][cols / 32]
   int n_chunk;           // tokens per unit: multiple of 16
+  int term_acc;          // 0: token terms stacked along N; 1: summed into the same columns
+  int max_bufs;          // accumulator sets wanted (1 or 2; the plan may give fewer)
   void* out;             // MODE 0: E4M3 terms of h [out_parts][pairs][rows]; MODE 1: fp32 [pairs][rows]
   uint8_t* out_scale;    // MODE 0: E8M0 of h [out_parts][pairs][rows / 32]
   int out_parts;
   float limit;
+  int prefetch;          // K-tiles of weights prefetched into L2 ahead of the loads (0: none)
   // filled in by mx_plan()
   int g;             // K-tiles per scale stage
   int acc_cols;      // TMEM columns per accumulator
+  int acc_bufs;      // accumulator sets
+  int tok_cols;      // TMEM columns of token scales per K-tile
+  int sf_kt;         // TMEM columns per K-tile in a scale stage (8 weight + tok_cols)
   int sf_stages;     // scale stages in TMEM
   int stages;        // shared-memory stages
   int stage_bytes;   // weights + token rows of one stage
+  int tma_scales;    // 1: E8M0 rows arrive by TMA in a shared-memory scale ring
+  int sc_slot_bytes; // one scale-ring slot: [2 x 128 weight rows + parts x n_chunk token rows][4 G]
+  int off_sc;        // scale ring
   int off_prefix;    // unit prefix + offsets copy
   int smem_bytes;
 };
@@ -99,30 +119,62 @@ struct MxArgs {
 // shape is outside what the kernel implements.
 inline bool mx_plan(MxArgs& a, int mode) {
   const int nc = a.n_chunk;
-  if (nc < 16 || nc % 16 || a.parts < 1 || a.parts > kMxMaxParts || a.parts * nc > kMxNMax) return false;
+  if (nc < 16 || nc % 16 || a.parts < 1 || a.parts > kMxMaxParts) return false;
+  if (a.term_acc != 0 && a.term_acc != 1) return false;
+  const int n = a.term_acc ? nc : a.parts * nc;  // the MMA's N
+  if (n > kMxNMax) return false;
   if (mode == 0 && (a.out_parts < 1 || a.out_parts > kMxMaxParts)) return false;
   if (a.cols % kMxKT || a.rows % (mode == 0 ? 128 : 256)) return false;
   // 16U4_ALIGN16B tensor maps: strides in multiples of 32 bytes
   if ((a.cols / 2) % 32 || a.expert_bytes % 32 || (a.cols / 32) % 4) return false;
   const int nkt = a.cols / kMxKT;
-  a.g = nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt % 2 == 0 ? 2 : 1;
-  const int n = a.parts * nc;
   a.acc_cols = (n + 31) / 32 * 32;
-  const int sf_cols = kMxSfPerKt * a.g;
-  a.sf_stages = (kTcTmemCols - 2 * a.acc_cols) / sf_cols;
+  a.tok_cols = a.term_acc ? 4 * a.parts : 4;
+  a.sf_kt = 8 + a.tok_cols;
+  // the most accumulator sets wanted that leave room for two scale stages,
+  // with the longest scale stage (G K-tiles) that does
+  a.g = 0;
+  const int want = a.max_bufs < 1 ? 1 : a.max_bufs < kMxMaxBufs ? a.max_bufs : kMxMaxBufs;
+  for (int nb = want; nb >= 1 && a.g == 0; --nb)
+    for (int G = 8; G >= 1 && a.g == 0; G /= 2)
+      if (nkt % G == 0 && (kTcTmemCols - nb * 2 * a.acc_cols) / (a.sf_kt * G) >= 2) {
+        a.g = G;
+        a.acc_bufs = nb;
+      }
+  if (a.g == 0) return false;
+  a.sf_stages = (kTcTmemCols - a.acc_bufs * 2 * a.acc_cols) / (a.sf_kt * a.g);
   if (a.sf_stages > kMxMaxSfStages) a.sf_stages = kMxMaxSfStages;
-  if (a.sf_stages < 1) return false;
-  a.stage_bytes = 2 * kMxTileBytes + n * 128;
+  a.stage_bytes = 2 * kMxTileBytes + a.parts * nc * 128;
   const int pre = (2 * (a.E + 1) * 4 + 127) / 128 * 128;
   const int budget = kTcSmemMax - 1024;
-  a.stages = (budget - pre) / a.stage_bytes;
+  // scale rows by TMA: rows of 4 G bytes, a multiple of 16, with row strides
+  // (cols / 32 bytes) a multiple of 16; otherwise the scale writers load them
+  a.tma_scales = (a.cols / 32) % 16 == 0 && a.g >= 4 ? 1 : 0;
+  a.sc_slot_bytes = a.tma_scales ? ((256 + a.parts * nc) * 4 * a.g + 127) / 128 * 128 : 0;
+  auto weight_stages = [&]() { return (budget - pre - a.sf_stages * a.sc_slot_bytes) / a.stage_bytes; };
+  a.stages = weight_stages();
+  while (a.tma_scales && a.stages < 4 && a.sf_stages > 2) {  // keep weight stages over scale slots
+    --a.sf_stages;
+    a.stages = weight_stages();
+  }
   if (a.stages > kMxMaxStages) a.stages = kMxMaxStages;
   if (a.stages < 2) return false;
-  a.off_prefix = a.stages * a.stage_bytes;
+  a.off_sc = a.stages * a.stage_bytes;
+  a.off_prefix = a.off_sc + a.sf_stages * a.sc_slot_bytes;
   a.smem_bytes = a.off_prefix + pre + 1024;
   // every CTA allocates all 512 TMEM columns, so no second CTA may share its
   // SM: more than half of the SM's shared memory guarantees that
   return a.smem_bytes <= kTcSmemMax && a.smem_bytes > kTcSmemMax / 2;
+}
+
+// Box {x, y, z} of a 3-D tensor map into L2 only (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+// Contiguous bytes into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both
@@ -165,6 +217,21 @@ __device__ __forceinline__ void load_words(const uint8_t* p, uint32_t* w) {
   }
 }
 
+// The same from shared memory (a generic pointer into it).
+template <int G>
+__device__ __forceinline__ void load_words_smem(const uint8_t* p, uint32_t* w) {
+  if constexpr (G >= 4) {
+#pragma unroll
+    for (int i = 0; i < G / 4; ++i) {
+      const uint4 a = reinterpret_cast<const uint4*>(p)[i];
+      w[4 * i] = a.x; w[4 * i + 1] = a.y; w[4 * i + 2] = a.z; w[4 * i + 3] = a.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < G; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  }
+}
+
 // E8M0 block scale of a group whose largest magnitude has fp32 bits `amax`:
 // 2^(floor(log2 amax) - 7), so every |v| / scale is below 256 and rounds to at
 // most 256, inside the E4M3 range (448); 2^-127 for groups under 2^-120 (and
@@ -185,11 +252,14 @@ __device__ __forceinline__ float e4m3_val(uint32_t code) {
 template <int MODE, int G>
 __global__ void __launch_bounds__(kMxThreads, 1)
     mx_expert_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap0,
-                     const __grid_constant__ CUtensorMap wmap1, const MxArgs args) {
+                     const __grid_constant__ CUtensorMap wmap1, const __grid_constant__ CUtensorMap smap0,
+                     const __grid_constant__ CUtensorMap smap1, const __grid_constant__ CUtensorMap tsmap,
+                     const MxArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[kMxMaxStages], empty[kMxMaxStages];
   __shared__ __align__(8) uint64_t sf_full[kMxMaxSfStages], sf_empty[kMxMaxSfStages];
-  __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
+  __shared__ __align__(8) uint64_t sc_full[kMxMaxSfStages], sc_empty[kMxMaxSfStages];
+  __shared__ __align__(8) uint64_t acc_full[kMxMaxBufs], acc_empty[kMxMaxBufs], mma_done;
   __shared__ uint32_t s_taddr;
   __shared__ int32_t s_abort;
 
@@ -204,10 +274,14 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   const int NC = args.n_chunk;
   const int P = args.parts;
   const int sr = args.cols / 32;  // E8M0 bytes per weight row and per token row
-  const uint32_t sf_base = 2 * args.acc_cols;
-  const int sf_cols = kMxSfPerKt * G;
+  const int NB = args.acc_bufs;
+  const bool summed = args.term_acc != 0;
+  const int TC = args.tok_cols;
+  const uint32_t sf_base = NB * 2 * args.acc_cols;
+  const int sf_cols = args.sf_kt * G;
 
   // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
+  griddep_wait();  // the offsets and token terms come from earlier kernels of the stream
   for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
   __syncthreads();
   if (warp == 0) {
@@ -235,9 +309,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     for (int s = 0; s < kMxMaxSfStages; ++s) {
       mbar_init(&sf_full[s], 4);  // one arrival per scale-writer warp
       mbar_init(&sf_empty[s], 1);
+      mbar_init(&sc_full[s], 1);
+      mbar_init(&sc_empty[s], 4);  // one arrival per scale-writer warp
     }
-    mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, 4);
+    for (int b = 0; b < kMxMaxBufs; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
     mbar_init(&mma_done, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -251,6 +329,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   tc_fence_after();
   const uint32_t tbase = s_taddr;
   const int n_units = s_prefix[E];
+  // the next kernel may begin launching once every CTA has started its last
+  // unit (its CTAs take an SM only as this kernel's CTAs leave)
+  if (tid == 0 && (int)blockIdx.x + (int)gridDim.x >= n_units) griddep_launch();
 
   // unit -> (expert, row tile, first grouped pair, tokens)
   auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
@@ -280,8 +361,34 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (lane == 0) {
       TcRing rs(args.stages);
       const uint64_t pol = policy_evict_first();
-      int issued = 0;
+      // L2 prefetch cursor, args.prefetch K-tiles ahead of the loads (across
+      // units): more HBM bytes in flight than the shared-memory ring holds.
+      // At a unit's first prefetch its E8M0 rows (contiguous per tile) go too.
+      const int64_t plane = (int64_t)args.rows * (args.cols / 2);
+      int pu = blockIdx.x, pkt = 0, pe = 0, pmt = 0, ppos = 0, pn = 0;
+      auto pf_step = [&]() {
+        if (pu >= n_units) return;
+        if (pkt == 0) {
+          decode_unit(pu, pe, pmt, ppos, pn);
+          const int r0 = MODE == 0 ? pmt * 128 : pmt * 256;
+          const uint32_t bytes = (uint32_t)((MODE == 0 ? 128 : 256) * sr);
+          l2_prefetch(args.w0 + (int64_t)pe * args.expert_bytes + plane + (int64_t)r0 * sr, bytes);
+          if (MODE == 0) l2_prefetch(args.w1 + (int64_t)pe * args.expert_bytes + plane + (int64_t)r0 * sr, bytes);
+        }
+        const int y0 = MODE == 0 ? pmt * 128 : pmt * 256;
+        const int y1 = MODE == 0 ? pmt * 128 : pmt * 256 + 128;
+        tma_prefetch_3d(&wmap0, pkt * kMxKT, y0, pe);
+        tma_prefetch_3d(MODE == 0 ? &wmap1 : &wmap0, pkt * kMxKT, y1, pe);
+        if (++pkt == nkt) {
+          pkt = 0;
+          pu += gridDim.x;
+        }
+      };
+      for (int i = 0; i < args.prefetch; ++i) pf_step();
+      int issued = 0, sc_issued = 0;
+      TcRing rc(args.sf_stages);  // scale-ring slots, one per scale stage
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         const int n16 = (n + 15) & ~15;  // rows past the chunk are loaded but never stored
@@ -290,6 +397,26 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const uint32_t tx = 2 * kMxTileTx + (uint32_t)(P * n16 * 128);
         bool ok = true;
         for (int kt = 0; kt < nkt; ++kt) {
+          if (args.tma_scales && kt % G == 0) {
+            // the scale stage's E8M0 rows: both weight tiles, then every term's
+            // token rows, [row][4 G bytes]
+            if (!mbar_wait(&sc_empty[rc.s], rc.ph ^ 1)) {
+              give_up();
+              ok = false;
+              break;
+            }
+            uint8_t* sd = smem + args.off_sc + rc.s * args.sc_slot_bytes;
+            const int xs = 4 * G * (kt / G);
+            mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * n16) * 4 * G));
+            tma_load_3d(sd, &smap0, xs, y0, e, &sc_full[rc.s], pol);
+            tma_load_3d(sd + 128 * 4 * G, MODE == 0 ? &smap1 : &smap0, xs, y1, e, &sc_full[rc.s], pol);
+            for (int p = 0; p < P; ++p)
+              for (int j = 0; j < n16; j += kTcBoxRows)
+                tma_load_2d(sd + (256 + p * n16 + j) * 4 * G, &tsmap, xs, p * args.pairs + pos0 + j, &sc_full[rc.s]);
+            rc.next();
+            ++sc_issued;
+          }
+          if (args.prefetch > 0) pf_step();
           if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
             give_up();
             ok = false;
@@ -313,6 +440,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const int s = (rs.s - 1 - i + rs.n) % rs.n;
         if (!mbar_wait(&full[s], s < rs.s ? rs.ph : rs.ph ^ 1)) set_error(kErrWaitTc);
       }
+      for (int i = 0; i < min(sc_issued, rc.n); ++i) {
+        const int s = (rc.s - 1 - i + rc.n) % rc.n;
+        if (!mbar_wait(&sc_full[s], s < rc.s ? rc.ph : rc.ph ^ 1)) set_error(kErrWaitTc);
+      }
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -321,12 +452,22 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       TcRing rs(args.stages), rf(args.sf_stages);
       uint32_t un = 0;
       bool ok = true;
+      // One thread issues every MMA, so the arithmetic between two MMAs is a
+      // dependent chain that nothing hides: descriptors are built once and
+      // advanced by adding byte offsets / 16 to their 14-bit address field
+      // (every operand lies below 256 KB, so the field never carries into the
+      // constant upper bits).
+      const uint64_t d_smem = sdesc_sw128(smem_u32(smem));
       for (int u = blockIdx.x; u < n_units && ok && !aborted(); u += gridDim.x, ++un) {
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         const int n16 = (n + 15) & ~15;
-        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, P * n16);
-        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) {
+        // summed terms: one MMA of N = tokens per term; stacked: one of N = P x tokens
+        const int nmma = summed ? P : 1;
+        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, summed ? n16 : P * n16);
+        const int b = (int)(un % (uint32_t)NB);
+        const uint32_t acc0 = tbase + (uint32_t)(b * 2 * args.acc_cols), acc1 = acc0 + args.acc_cols;
+        if (!mbar_wait(&acc_empty[b], ((un / NB) & 1) ^ 1)) {
           give_up();
           break;
         }
@@ -342,18 +483,25 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t wa = smem_u32(smem + rs.s * args.stage_bytes), ba = wa + 2 * kMxTileBytes;
+          // this stage's operands: weight tiles at 0 and 16 KB, token rows at 32 KB
+          // (term p's n16 rows p * n16 * 128 bytes further); a k-block is 32 bytes
+          const uint64_t da0 = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
+          const uint64_t da1 = da0 + (kMxTileBytes >> 4), db = da0 + (2 * kMxTileBytes >> 4);
           const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
+          const uint32_t sfa0 = sfc + 8 * j, sfa1 = sfa0 + 4, sfb0 = sfc + 8 * G + TC * j;
+          const uint32_t first = kt > 0 ? 1u : 0u;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
             const uint32_t sel = (uint32_t)kb << 30;
-            const uint64_t bd = sdesc_sw128(ba + kb * 32);
-            const uint32_t sfb = (sfc + 8 * G + 4 * j) | sel;
-            const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-            umma_mx(tbase, sdesc_sw128(wa + kb * 32), bd, id, acc, (sfc + 8 * j) | sel, sfb);
-            umma_mx(tbase + args.acc_cols, sdesc_sw128(wa + kMxTileBytes + kb * 32), bd, id, acc,
-                    (sfc + 8 * j + 4) | sel, sfb);
+            const uint64_t ko = (uint64_t)(2 * kb);
+            for (int p = 0; p < nmma; ++p) {
+              const uint64_t bd = db + ko + (uint64_t)((p * n16 * 128) >> 4);
+              const uint32_t sfb = (sfb0 + 4 * p) | sel;
+              const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
+              umma_mx(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
+              umma_mx(acc1, da1 + ko, bd, id, acc, sfa1 | sel, sfb);
+            }
           }
           umma_commit(&empty[rs.s]);
           rs.next();
@@ -361,7 +509,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             umma_commit(&sf_empty[rf.s]);
             rf.next();
           }
-          if (kt == nkt - 1) umma_commit(&acc_full);
+          if (kt == nkt - 1) umma_commit(&acc_full[b]);
         }
       }
       if (!ok) give_up();
@@ -382,32 +530,60 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const int n16 = (n + 15) & ~15;
       bool ok = true;
       for (int g = 0; g < nkt / G; ++g) {
+        // the stage's E8M0 rows: from the scale ring (TMA) or straight from memory
+        const uint8_t* ss = nullptr;
+        if (args.tma_scales) {
+          if (!warp_wait(&sc_full[rf.s], rf.ph)) {
+            ok = false;
+            break;
+          }
+          ss = smem + args.off_sc + rf.s * args.sc_slot_bytes;
+        }
         // weight scales: a[8 j + 4 m + c] = bytes 4 (G g + j) .. +3 of row 32 c + lane of tile m
         uint32_t a[8 * G], b[4 * G];
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int R = MODE == 0 ? mt * 128 + 32 * c + lane : mt * 256 + 128 * m + 32 * c + lane;
-            const uint8_t* src = (MODE == 0 && m == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes + plane +
-                                 (int64_t)R * sr + 4 * G * g;
             uint32_t w[G];
-            load_words<G>(src, w);
+            if (ss != nullptr) {
+              load_words_smem<G>(ss + (128 * m + 32 * c + lane) * 4 * G, w);
+            } else {
+              const int R = MODE == 0 ? mt * 128 + 32 * c + lane : mt * 256 + 128 * m + 32 * c + lane;
+              load_words<G>((MODE == 0 && m == 1 ? args.w1 : args.w0) + (int64_t)e * args.expert_bytes + plane +
+                                (int64_t)R * sr + 4 * G * g,
+                            w);
+            }
 #pragma unroll
             for (int j = 0; j < G; ++j) a[8 * j + 4 * m + c] = w[j];
           }
-        // token scales: b[4 j + c] for N index 32 c + lane = term p, token t
+        // token scales, 4 columns at a time: stacked, column c holds N index
+        // 32 c + lane (term nn / n16, token nn mod n16); summed, block p of 4
+        // columns holds term p, column c of it token 32 c + lane
+        auto load_tokens = [&](int q4) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int nn = 32 * c + lane, p = nn / n16, t = nn - p * n16;
-          uint32_t w[G];
+          for (int c = 0; c < 4; ++c) {
+            int p, t;
+            if (summed) {
+              p = q4;
+              t = 32 * c + lane;
+            } else {
+              const int nn = 32 * c + lane;
+              p = nn / n16;
+              t = nn - p * n16;
+            }
+            uint32_t w[G];
 #pragma unroll
-          for (int j = 0; j < G; ++j) w[j] = 0;
-          if (p < P && t < n)
-            load_words<G>(args.b_scale + ((int64_t)p * args.pairs + pos0 + t) * sr + 4 * G * g, w);
+            for (int j = 0; j < G; ++j) w[j] = 0;
+            if (p < P && t < n) {
+              if (ss != nullptr) load_words_smem<G>(ss + (256 + p * n16 + t) * 4 * G, w);
+              else load_words<G>(args.b_scale + ((int64_t)p * args.pairs + pos0 + t) * sr + 4 * G * g, w);
+            }
 #pragma unroll
-          for (int j = 0; j < G; ++j) b[4 * j + c] = w[j];
-        }
+            for (int j = 0; j < G; ++j) b[4 * j + c] = w[j];
+          }
+        };
+        load_tokens(0);  // in flight with the weight scales while the stage frees up
         if (!warp_wait(&sf_empty[rf.s], rf.ph ^ 1)) {
           ok = false;
           break;
@@ -416,18 +592,25 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const uint32_t col = tbase + lrow + sf_base + rf.s * sf_cols;
 #pragma unroll
         for (int i = 0; i < G; ++i) tmem_st8(col + 8 * i, a + 8 * i);
-        if constexpr (G == 1) {  // 4 token-scale columns
-          asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(col + 8), "r"(b[0]),
-                       "r"(b[1]), "r"(b[2]), "r"(b[3])
-                       : "memory");
-        } else {
+        for (int q4 = 0; q4 < TC / 4; ++q4) {
+          if (q4 > 0) {
+            tmem_st_wait();  // the previous group's registers are stored before b is refilled
+            load_tokens(q4);
+          }
 #pragma unroll
-          for (int i = 0; i < G / 2; ++i) tmem_st8(col + 8 * G + 8 * i, b + 8 * i);
+          for (int j = 0; j < G; ++j)
+            asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             col + 8 * G + TC * j + 4 * q4),
+                         "r"(b[4 * j]), "r"(b[4 * j + 1]), "r"(b[4 * j + 2]), "r"(b[4 * j + 3])
+                         : "memory");
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_full[rf.s]);
+        if (lane == 0) {
+          mbar_arrive(&sf_full[rf.s]);
+          if (ss != nullptr) mbar_arrive(&sc_empty[rf.s]);  // every read of the slot is done
+        }
         rf.next();
       }
       if (!ok) {
@@ -444,19 +627,22 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
       const int n16 = (n + 15) & ~15;
-      if (!warp_wait(&acc_full, un & 1)) {
+      const int b = (int)(un % (uint32_t)NB);
+      const uint32_t accb = tbase + lrow + (uint32_t)(b * 2 * args.acc_cols);
+      if (!warp_wait(&acc_full[b], (un / NB) & 1)) {
         give_up();
         break;
       }
       tc_fence_after();
+      const int pe = summed ? 1 : P;  // stacked terms are summed here
       for (int c0 = 0; c0 < n; c0 += 16) {
         float g[16], v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) g[j] = v[j] = 0.f;
-        for (int p = 0; p < P; ++p) {  // sum of the token terms
+        for (int p = 0; p < pe; ++p) {
           uint32_t t0[16], t1[16];
-          tmem_ld16(tbase + lrow + p * n16 + c0, t0);
-          tmem_ld16(tbase + lrow + args.acc_cols + p * n16 + c0, t1);
+          tmem_ld16(accb + p * n16 + c0, t0);
+          tmem_ld16(accb + args.acc_cols + p * n16 + c0, t1);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -497,7 +683,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty);
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
 
@@ -515,6 +701,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 __global__ void gather_split_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int top_k,
                                     int hidden, int64_t pairs, int parts, uint8_t* __restrict__ q,
                                     uint8_t* __restrict__ sc) {
+  griddep_wait();
   const int h8 = hidden / 8;
   const int64_t n = pairs * h8;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;

@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(
   extern __shared__ int32_t hist[];  // [32 warps][E]
   __shared__ int32_t scan_buf[kPermuteThreads];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();
+  griddep_launch();
   for (int i = tid; i < 32 * E; i += kPermuteThreads) hist[i] = 0;
   __syncthreads();
 

@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(kLogitThreads) route_logits_kernel(const __nv_
                                                                      const float* __restrict__ wr, int E,
                                                                      float* __restrict__ logits) {
   extern __shared__ float4 s_w4[];  // [kLogitExperts][H / 4]
+  griddep_wait();
+  griddep_launch();
   const int e0 = blockIdx.x * kLogitExperts;
   const int ne = min(kLogitExperts, E - e0);
   const int h4 = H / 4, h8 = H / 8;
@@ -98,6 +100,8 @@ __global__ void __launch_bounds__(128) route_select_kernel(
     float* __restrict__ topk_w) {
   extern __shared__ float s_sm[];  // [4][E]
   __shared__ int32_t sel[4][32];
+  griddep_wait();
+  griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + warp;
   if (t >= T) return;

@@ -47,6 +47,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 template <int MODE>
 __global__ void __launch_bounds__(kShThreads) shared_decode_kernel(const ShArgs args) {
   __shared__ float s_red[kShWarps][32][4];
+  griddep_wait();
+  griddep_launch();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int I_or_H = args.rows;

@@ -329,6 +329,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
   // The group offsets are read once, by all threads in parallel, into shared
   // memory: the scan and every unit lookup then stay on chip.
+  griddep_wait();  // inputs come from earlier kernels of the stream
   if (grouped)
     for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
   __syncthreads();
@@ -375,6 +376,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   tc_fence_after();
   const uint32_t tbase = s_taddr;
   const int n_units = s_prefix[E];
+  // the next kernel may begin launching once every CTA has started its last unit
+  if (tid == 0 && (int)blockIdx.x + (int)gridDim.x >= n_units) griddep_launch();
 
   // unit -> (group, row tile, first row of the token matrix, tokens)
   auto decode_unit = [&](int u, int& e, int& mt, int& pos0, int& n) {
@@ -571,6 +574,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       const int n_slots = nst / args.st_per_slot;
       int issued = 0;
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+        if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         bool ok = true;
@@ -648,6 +652,9 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     if (lane == 0) {
       TcRing rs(args.stages);
       uint32_t un = 0;
+      // descriptors built once, advanced by byte offset / 16 (operands lie
+      // below 256 KB: the 14-bit address field never carries)
+      const uint64_t d_b = sdesc_sw128(smem_u32(s_b));
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
@@ -667,16 +674,19 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
             break;
           }
           tc_fence_after();
-          const uint32_t bsa = smem_u32(s_b + rs.s * bst);
+          const uint64_t bd0 = d_b + (uint64_t)((rs.s * bst) >> 4);
           const uint32_t a0 = tbase + a_base + rs.s * kTcStageCols;
+          const uint32_t acc1 = tbase + args.acc_cols;
+          const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
           for (int g = 0; g < kTcKG; ++g) {
+            const uint64_t bdg = bd0 + (uint64_t)((g * atom) >> 4);
 #pragma unroll
             for (int ks = 0; ks < kTcKB / 16; ++ks) {
-              const uint64_t bd = sdesc_sw128(bsa + g * atom + ks * 32);
-              const uint32_t acc = (st > 0 || g > 0 || ks > 0) ? 1u : 0u;
+              const uint64_t bd = bdg + (uint64_t)(2 * ks);
+              const uint32_t acc = (g > 0 || ks > 0) ? 1u : first;
               umma_tmem_a(tbase, a0 + g * 64 + ks * 8, bd, idesc, acc);
-              umma_tmem_a(tbase + args.acc_cols, a0 + g * 64 + 32 + ks * 8, bd, idesc, acc);
+              umma_tmem_a(acc1, a0 + g * 64 + 32 + ks * 8, bd, idesc, acc);
             }
           }
           umma_commit(&empty[rs.s]);
@@ -770,6 +780,7 @@ __device__ __forceinline__ bool f16x2_has_inf(uint32_t h) {
 // inf and the call records device error 0x303.
 __global__ void gather_f16_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int K, int h8,
                                   int64_t rows, uint4* __restrict__ out) {
+  griddep_wait();
   const int64_t n = rows * h8;
   bool inf = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
@@ -788,6 +799,7 @@ __global__ void gather_f16_kernel(const uint4* __restrict__ x, const int32_t* __
 // each difference is exact in fp32.  Laid out [rows][3 * cols]: hi | mid | lo.
 __global__ void split3_bf16_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ out, int rows,
                                    int cols) {
+  griddep_wait();
   const int64_t n = (int64_t)rows * cols;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t rr = i / cols, c = i % cols;

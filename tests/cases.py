@@ -49,7 +49,8 @@ class Case:
 def make_case(dims: gen.Dims, T: int, seed: int = 0, layer: int = 0, bias=None, hashed: bool = False,
               vocab: int = gen.HASH_VOCAB, with_shared: bool = True, e_range=None, x_edit=None) -> Case:
     """A seeded case.  e_range: (lo, hi) E8M0 exponents of the routed weights
-    (default [118, 124]).  x_edit(t, row_bits) -> row_bits: applied to every
+    (default [118, 124]), or (lo, hi, row_span): a base per weight row in
+    [lo, hi - row_span] plus [0, row_span] per group.  x_edit(t, row_bits) -> row_bits: applied to every
     drawn activation row (and to every redraw) before routing, to shape edge
     cases such as outlier channels or all-zero groups."""
     H, I, E, K = dims.hidden, dims.inter, dims.n_experts, dims.top_k

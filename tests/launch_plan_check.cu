@@ -33,15 +33,35 @@ static moe_mxfp4_proj proj(uintptr_t base, int rows, int cols) {
 }
 
 static void check_mx_plan(const MxArgs& a, int mode, const char* name, int T) {
-  const int n = a.parts * a.n_chunk;
+  const int n = a.term_acc ? a.n_chunk : a.parts * a.n_chunk;  // the MMA's N
+  CHECK(a.term_acc == 0 || a.term_acc == 1, "%s T=%d layout", name, T);
   CHECK(n <= kMxNMax && n % 16 == 0, "%s T=%d N=%d", name, T, n);
-  CHECK(a.acc_cols >= n, "%s T=%d", name, T);
-  CHECK(2 * a.acc_cols + a.sf_stages * kMxSfPerKt * a.g <= kTcTmemCols, "%s T=%d TMEM", name, T);
-  CHECK(a.sf_stages >= 1 && a.stages >= 2, "%s T=%d rings", name, T);
+  CHECK(a.acc_cols >= n && a.acc_cols % 32 == 0, "%s T=%d", name, T);
+  CHECK(a.acc_bufs >= 1 && a.acc_bufs <= kMxMaxBufs && a.acc_bufs <= (a.max_bufs > 1 ? a.max_bufs : 1),
+        "%s T=%d accumulator sets", name, T);
+  // token scales: stacked, N <= 128 indices in 4 columns; summed, 4 columns
+  // (128 tokens) per term; each term block starts on a multiple of 4
+  CHECK(a.tok_cols == (a.term_acc ? 4 * a.parts : 4) && a.sf_kt == 8 + a.tok_cols, "%s T=%d scale cols", name, T);
+  CHECK(a.term_acc ? a.n_chunk <= 128 : a.parts * a.n_chunk <= 128, "%s T=%d scale coverage", name, T);
+  CHECK(a.acc_bufs * 2 * a.acc_cols + a.sf_stages * a.sf_kt * a.g <= kTcTmemCols, "%s T=%d TMEM", name, T);
+  CHECK(a.sf_stages >= 2 && a.sf_stages <= kMxMaxSfStages && a.stages >= 2, "%s T=%d rings", name, T);
   CHECK((a.cols / kMxKT) % a.g == 0, "%s T=%d G", name, T);
   CHECK(a.stage_bytes % 1024 == 0, "%s T=%d stage", name, T);
-  CHECK(a.stage_bytes >= 2 * kMxTileBytes + n * 128, "%s T=%d stage size", name, T);
-  CHECK(a.off_prefix == a.stages * a.stage_bytes, "%s T=%d prefix", name, T);
+  CHECK(a.stage_bytes >= 2 * kMxTileBytes + a.parts * a.n_chunk * 128, "%s T=%d stage size", name, T);
+  // shared memory: weight stages, then the scale ring (TMA-fed E8M0 rows),
+  // then the unit prefix and offsets copy
+  CHECK(a.off_sc == a.stages * a.stage_bytes, "%s T=%d scale ring offset", name, T);
+  CHECK(a.off_prefix == a.off_sc + a.sf_stages * a.sc_slot_bytes, "%s T=%d prefix", name, T);
+  if (a.tma_scales) {
+    // a slot holds both weight tiles' 128 rows and every term's n_chunk token
+    // rows of 4 G bytes; TMA rows are 16-byte multiples with 16-byte strides
+    CHECK(a.sc_slot_bytes >= (256 + a.parts * a.n_chunk) * 4 * a.g && a.sc_slot_bytes % 128 == 0,
+          "%s T=%d scale slot", name, T);
+    CHECK(a.g >= 4 && (4 * a.g) % 16 == 0 && (a.cols / 32) % 16 == 0, "%s T=%d scale boxes", name, T);
+    CHECK(a.off_sc % 1024 == 0, "%s T=%d scale ring alignment", name, T);
+  } else {
+    CHECK(a.sc_slot_bytes == 0, "%s T=%d scale slot without TMA", name, T);
+  }
   CHECK(a.off_prefix + 2 * (a.E + 1) * 4 + 1024 <= a.smem_bytes, "%s T=%d prefix room", name, T);
   CHECK(a.smem_bytes <= kTcSmemMax && 2 * a.smem_bytes > kTcSmemMax, "%s T=%d smem %d", name, T, a.smem_bytes);
   CHECK(a.rows % (mode == 0 ? 128 : 256) == 0, "%s T=%d rows", name, T);

@@ -82,6 +82,10 @@ def test_device_generator_matches_host():
     gen.mxfp4_fill_device(buf.data_ptr(), torch.cuda.current_stream().cuda_stream, 0, 0, "up", 2, I, H)
     b = buf.cpu().numpy()
     assert np.array_equal(b[eb4:], gen.mxfp4_expert_host(0, 0, "up", 1, I, H))
+    # per-row exponent bases (the edge-case weights)
+    gen.mxfp4_fill_device(buf.data_ptr(), torch.cuda.current_stream().cuda_stream, 3, 1, "down", 2, H, I, 0, 230, 6)
+    b = buf.cpu().numpy()
+    assert np.array_equal(b[eb4:], gen.mxfp4_expert_host(3, 1, "down", 1, H, I, 0, 230, 6))
 
 
 # ---- routing ------------------------------------------------------------------

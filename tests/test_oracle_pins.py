@@ -319,3 +319,17 @@ def test_layer_missing_expert_blob_is_an_error(oracle_lib):
     wr = gen.router_weight(0, 0, d.n_experts, d.hidden)
     with pytest.raises(ValueError):
         oracle_lib.moe_layer(d, x, np.arange(2), wr, None, {}, {}, {}, nthreads=1)
+
+
+def test_generator_row_bases():
+    """The per-row exponent mode: every row's bytes lie within row_span of a
+    base in [lo, hi - row_span], and the bases cover the range."""
+    rows, cols = 64, 256
+    blob = gen.mxfp4_expert_host(5, 0, "down", 3, rows, cols, 0, 230, 6)
+    sc = blob[rows * cols // 2:].reshape(rows, cols // 32).astype(int)
+    assert (sc.max(1) - sc.min(1) <= 6).all()
+    assert sc.min() >= 0 and sc.max() <= 230
+    assert sc.min(1).max() - sc.min(1).min() > 100  # bases spread over the range
+    # the default mode is unchanged by the new parameter
+    assert np.array_equal(gen.mxfp4_expert_host(5, 0, "down", 3, rows, cols),
+                          gen.mxfp4_expert_host(5, 0, "down", 3, rows, cols, gen.E8M0_LO, gen.E8M0_HI, -1))

@@ -12,7 +12,10 @@ import os
 from dataclasses import dataclass
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIBRARY=debug selects libmoe_debug.so: the same kernels built with
+# bounds checks on the indices they otherwise trust (moe_device_error()
+# reports 0x501 / 0x502 instead of an out-of-bounds access).
+LIB_PATH = os.path.join(_HERE, "libmoe_debug.so" if os.environ.get("MOE_LIBRARY") == "debug" else "libmoe.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_UNSUPPORTED",
@@ -142,6 +145,8 @@ DEVICE_ERR_WAIT_TC = 0x301
 DEVICE_ERR_SPAN_FLUSH = 0x302
 DEVICE_ERR_F16_RANGE = 0x303
 DEVICE_ERR_WAIT_SELFTEST = 0x401
+DEVICE_ERR_BAD_INDEX = 0x501     # debug build only
+DEVICE_ERR_BAD_OFFSETS = 0x502   # debug build only
 
 
 def moe_selftest_wait(wait_us: int, stream=None):

@@ -23,12 +23,16 @@ def _stale(target: str, sources) -> bool:
     return any(os.path.getmtime(s) > t for s in sources)
 
 
-def build_libmoe(force: bool = False) -> str:
-    out = os.path.join(PKG, "libmoe.so")
+def build_libmoe(force: bool = False, debug: bool = False) -> str:
+    """libmoe.so, or with debug=True libmoe_debug.so: the same library built
+    with -DMOE_DEBUG, whose kernels check the indices they otherwise trust and
+    report a bad one through moe_device_error() instead of touching memory
+    out of bounds."""
+    out = os.path.join(PKG, "libmoe_debug.so" if debug else "libmoe.so")
     srcs = glob.glob(os.path.join(PKG, "csrc", "*")) + [os.path.join(ROOT, "include", "moe.h")]
     if force or _stale(out, srcs):
-        cmd = [NVCC, *ARCH, *FLAGS, "-I", os.path.join(ROOT, "include"), os.path.join(PKG, "csrc", "moe.cu"),
-               "-o", out]
+        cmd = [NVCC, *ARCH, *FLAGS, *(["-DMOE_DEBUG"] if debug else []), "-I", os.path.join(ROOT, "include"),
+               os.path.join(PKG, "csrc", "moe.cu"), "-o", out]
         subprocess.check_call(cmd)
     return out
 
@@ -43,6 +47,7 @@ def build_gen(force: bool = False) -> str:
 
 def build_all(force: bool = False) -> None:
     build_libmoe(force)
+    build_libmoe(force, debug=True)
     build_gen(force)
 
 

@@ -26,6 +26,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
   for (int k = 0; k < K; ++k) {
     const int64_t pos = inv[(int64_t)t * K + k];
     const float wk = w[(int64_t)t * K + k];
+    if (kDebug && (pos < 0 || pos >= (int64_t)gridDim.y * K)) {  // gridDim.y = T
+      set_error(kErrBadIndex);
+      continue;
+    }
     const float4 y = __ldg(reinterpret_cast<const float4*>(y_perm + pos * H) + c4);
     acc.x = fmaf(wk, y.x, acc.x);
     acc.y = fmaf(wk, y.y, acc.y);

@@ -20,7 +20,18 @@ enum : int32_t {
   kErrSpanFlush = 0x302,    // a weight row's E8M0 bytes span > 36 octaves: the lowest groups were flushed
   kErrF16Range = 0x303,     // an activation beyond the f16 range reached the dequantising expert path
   kErrWaitSelftest = 0x401, // moe_selftest_wait: its wait ran out, as it should
+  kErrBadIndex = 0x501,     // debug build: a pair index (perm / inv) outside [0, T * top_k)
+  kErrBadOffsets = 0x502,   // debug build: group offsets not non-decreasing from 0 to T * top_k
 };
+
+// The debug build (-DMOE_DEBUG) checks the indices the kernels otherwise
+// trust -- the grouped pair ids, the group offsets, the combine's slots --
+// records kErrBadIndex / kErrBadOffsets and skips the access instead.
+#ifdef MOE_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
 
 __device__ int32_t g_error;
 

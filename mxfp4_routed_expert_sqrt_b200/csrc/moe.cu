@@ -50,11 +50,14 @@ moe_status launch_status() {
   return MOE_OK;
 }
 
-// Kernels are launched with programmatic stream serialization: each one may
-// begin (its prologue: barriers, TMEM, descriptor fetches) while its
-// predecessor in the stream finishes, and waits in griddep_wait() before its
-// first global access, so stream order holds for every byte.
-constexpr bool kUsePdl = true;
+// Programmatic stream serialization: with it, each kernel may begin (its
+// prologue: barriers, TMEM, descriptor fetches) while its predecessor in the
+// stream finishes, and waits in griddep_wait() before its first global
+// access, so stream order holds for every byte.  Measured on one B200 (decode
+// layer passes, interleaved A/B in CUDA graphs): no gain in the expert call
+// and ~1.5% slower whole layers, so it is off; the kernels keep their waits
+// (no-ops without the attribute).
+constexpr bool kUsePdl = false;
 
 template <typename... KArgs, typename... Args>
 moe_status launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -94,15 +97,16 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Row-major 16-bit [rows][cols] viewed by TMA with a {64, 16} box and 128-byte
-// swizzle (the token-operand layout of the tensor-core expert kernel).
-bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+// Row-major 16-bit [rows][cols] viewed by TMA with a {64, box_rows} box (one
+// k-block of a unit's n_chunk token rows) and 128-byte swizzle (the
+// token-operand layout of the tensor-core expert kernel).
+bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows,
                   CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kTcBoxRows};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -172,54 +176,58 @@ moe_status launch_tc(const CUtensorMap& bmap, const TcArgs& a, cudaStream_t s) {
 }
 
 // E2M1 plane of an MXFP4 weight array viewed by the block-scaled expert
-// kernel's loader: {columns (codes), rows, experts}, 128 x 128 boxes widened to
-// the f8f6f4 shared-memory layout (16U4_ALIGN16B), 128-byte swizzle.
-bool make_mx_weight_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a) {
+// kernel's loader: {columns (codes), rows, experts}, boxes of 128 codes x
+// box_rows rows (128: one tile; 256: both tiles of a down unit) widened to the
+// f8f6f4 shared-memory layout (16U4_ALIGN16B), 128-byte swizzle.
+bool make_mx_weight_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a, int box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr || base == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)a.cols, (cuuint64_t)a.rows, (cuuint64_t)a.E};
   cuuint64_t strides[2] = {(cuuint64_t)a.cols / 2, (cuuint64_t)a.expert_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)kMxKT, 128, 1}, estr[3] = {1, 1, 1};
+  cuuint32_t box[3] = {(cuuint32_t)kMxKT, (cuuint32_t)box_rows, 1}, estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E4M3 token terms [rows][cols] bytes with a {128, 16} box, 128-byte swizzle.
-bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t cols) {
+// E4M3 token terms [parts][pairs][cols] bytes viewed as {cols, pairs, parts}
+// with one {128, n_chunk, parts} box per stage (every term's rows of a unit in
+// one copy), 128-byte swizzle.
+bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t pairs, int parts, int64_t cols, int n_chunk) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols};
-  cuuint32_t box[2] = {(cuuint32_t)kMxKT, (cuuint32_t)kTcBoxRows}, estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)pairs, (cuuint64_t)parts};
+  cuuint64_t strides[2] = {(cuuint64_t)cols, (cuuint64_t)(cols * pairs)};
+  cuuint32_t box[3] = {(cuuint32_t)kMxKT, (cuuint32_t)n_chunk, (cuuint32_t)parts}, estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // E8M0 plane of an MXFP4 weight array: {row bytes (cols / 32), rows, experts}
-// with boxes of one scale stage's bytes (4 G) of 128 rows, no swizzle.
-bool make_mx_scale_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a) {
+// with boxes of one scale stage's bytes (4 G) of box_rows rows, no swizzle.
+bool make_mx_scale_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a, int box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr || base == nullptr) return false;
   const int64_t plane = (int64_t)a.rows * (a.cols / 2);
   cuuint64_t dims[3] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.rows, (cuuint64_t)a.E};
   cuuint64_t strides[2] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.expert_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)(4 * a.g), 128, 1}, estr[3] = {1, 1, 1};
+  cuuint32_t box[3] = {(cuuint32_t)(4 * a.g), (cuuint32_t)box_rows, 1}, estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base + plane), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E8M0 scales of the token terms [parts * pairs][cols / 32] with boxes of one
-// scale stage's bytes of 16 rows, no swizzle.
+// E8M0 scales of the token terms [parts][pairs][cols / 32] viewed as
+// {cols / 32, pairs, parts} with one {4 G, n_chunk, parts} box per scale
+// stage, no swizzle.
 bool make_token_scale_map(CUtensorMap* map, const MxArgs& a) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr || a.b_scale == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.parts * a.pairs};
-  cuuint64_t strides[1] = {(cuuint64_t)a.cols / 32};
-  cuuint32_t box[2] = {(cuuint32_t)(4 * a.g), (cuuint32_t)kTcBoxRows}, estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.b_scale), dims, strides, box, estr,
+  cuuint64_t dims[3] = {(cuuint64_t)a.cols / 32, (cuuint64_t)a.pairs, (cuuint64_t)a.parts};
+  cuuint64_t strides[2] = {(cuuint64_t)a.cols / 32, (cuuint64_t)(a.cols / 32) * a.pairs};
+  cuuint32_t box[3] = {(cuuint32_t)(4 * a.g), (cuuint32_t)a.n_chunk, (cuuint32_t)a.parts}, estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a.b_scale), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -230,16 +238,17 @@ moe_status launch_mx_g(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s)
   static std::atomic<uint64_t> configured{0};
   if (!smem_limit_once(configured, mx_expert_kernel<MODE, G>, kTcSmemMax)) return MOE_ERR_CUDA;
   CUtensorMap w0, w1, s0, s1, ts;
-  if (!make_mx_weight_map(&w0, a.w0, a)) return MOE_ERR_CUDA;
+  const int box_rows = MODE == 0 ? 128 : 256;  // MODE 1: both 128-row tiles of a unit in one box
+  if (!make_mx_weight_map(&w0, a.w0, a, box_rows)) return MOE_ERR_CUDA;
   if (MODE == 0) {
-    if (!make_mx_weight_map(&w1, a.w1, a)) return MOE_ERR_CUDA;
+    if (!make_mx_weight_map(&w1, a.w1, a, box_rows)) return MOE_ERR_CUDA;
   } else {
     w1 = w0;
   }
   if (a.tma_scales) {
-    if (!make_mx_scale_map(&s0, a.w0, a) || !make_token_scale_map(&ts, a)) return MOE_ERR_CUDA;
+    if (!make_mx_scale_map(&s0, a.w0, a, box_rows) || !make_token_scale_map(&ts, a)) return MOE_ERR_CUDA;
     if (MODE == 0) {
-      if (!make_mx_scale_map(&s1, a.w1, a)) return MOE_ERR_CUDA;
+      if (!make_mx_scale_map(&s1, a.w1, a, box_rows)) return MOE_ERR_CUDA;
     } else {
       s1 = s0;
     }
@@ -414,7 +423,7 @@ moe_status moe_route(const moe_dims* dims, const void* x, int32_t T, const float
     if ((st = launch_k(split3_bf16_kernel, dim3(2 * sm_count()), dim3(256), 0, s, router_w, split, E, H)) != MOE_OK)
       return st;
     CUtensorMap xmap;
-    if (!make_row_map(&xmap, x, T, H)) return MOE_ERR_CUDA;
+    if (!make_row_map(&xmap, x, T, H, 32)) return MOE_ERR_CUDA;
     TcArgs a{};
     a.w0 = reinterpret_cast<const uint8_t*>(split);
     a.rows = E;
@@ -501,7 +510,8 @@ moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t
                            L.xq, L.xs);
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
-  if (!make_term_map(&xmap, L.xq, kXTerms * L.pairs, H) || !make_term_map(&hmap, L.hq, kHTerms * L.pairs, I))
+  if (!make_term_map(&xmap, L.xq, L.pairs, kXTerms, H, L.g.n_chunk) ||
+      !make_term_map(&hmap, L.hq, L.pairs, kHTerms, I, L.d.n_chunk))
     return MOE_ERR_CUDA;
   if ((st = launch_mx<0>(xmap, L.g, s)) != MOE_OK) return st;
   return launch_mx<1>(hmap, L.d, s);
@@ -522,8 +532,8 @@ moe_status expert_gemm_dequant(const moe_dims* dims, const void* x, int32_t T, c
                            reinterpret_cast<uint4*>(L.x16));
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
-  if (!make_row_map(&xmap, L.x16, L.pairs, H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_row_map(&hmap, L.h16, L.pairs, I, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+  if (!make_row_map(&xmap, L.x16, L.pairs, H, L.g.n_chunk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_row_map(&hmap, L.h16, L.pairs, I, L.d.n_chunk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   if ((st = launch_tc<0, kAMxfp4>(xmap, L.g, s)) != MOE_OK) return st;
   return launch_tc<1, kAMxfp4>(hmap, L.d, s);
@@ -577,7 +587,7 @@ moe_status shared_expert(const moe_dims* dims, const void* x, int32_t T, const v
     // below 16 significant bits
     __nv_bfloat16* h2 = static_cast<__nv_bfloat16*>(ws);
     CUtensorMap xmap, hmap;
-    if (!make_row_map(&xmap, x, T, H) || !make_row_map(&hmap, h2, T, 2 * I)) return MOE_ERR_CUDA;
+    if (!make_row_map(&xmap, x, T, H, kTcNMax) || !make_row_map(&hmap, h2, T, 2 * I, kTcNMax)) return MOE_ERR_CUDA;
     TcArgs g{};
     g.w0 = static_cast<const uint8_t*>(wg);
     g.w1 = static_cast<const uint8_t*>(wu);

@@ -167,6 +167,16 @@ inline bool mx_plan(MxArgs& a, int mode) {
   return a.smem_bytes <= kTcSmemMax && a.smem_bytes > kTcSmemMax / 2;
 }
 
+// Box {x, y, z} of a 3-D tensor map into shared memory (no cache hint).
+__device__ __forceinline__ void tma_load_3d_nohint(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                                   uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Box {x, y, z} of a 3-D tensor map into L2 only (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
@@ -284,6 +294,16 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   griddep_wait();  // the offsets and token terms come from earlier kernels of the stream
   for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
   __syncthreads();
+  if (kDebug) {  // offsets must run from 0 to the pair count without decreasing
+    bool bad = false;
+    for (int i = tid; i < E; i += blockDim.x) bad |= s_off[i] > s_off[i + 1];
+    if (tid == 0) bad |= s_off[0] != 0 || s_off[E] != args.pairs;
+    if (__syncthreads_or(bad ? 1 : 0)) {
+      if (tid == 0) set_error(kErrBadOffsets);
+      for (int i = tid; i <= E; i += blockDim.x) s_off[i] = 0;  // no units
+      __syncthreads();
+    }
+  }
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < E; base += 32) {
@@ -391,10 +411,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
-        const int n16 = (n + 15) & ~15;  // rows past the chunk are loaded but never stored
+        (void)n;
         const int y0 = MODE == 0 ? mt * 128 : mt * 256;
-        const int y1 = MODE == 0 ? mt * 128 : mt * 256 + 128;
-        const uint32_t tx = 2 * kMxTileTx + (uint32_t)(P * n16 * 128);
+        // one stage: both weight tiles (MODE 1: one 256-row box) and one box of
+        // every term's n_chunk token rows (rows past the unit's tokens are
+        // loaded but never stored)
+        const uint32_t tx = 2 * kMxTileTx + (uint32_t)(P * NC * 128);
         bool ok = true;
         for (int kt = 0; kt < nkt; ++kt) {
           if (args.tma_scales && kt % G == 0) {
@@ -407,12 +429,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             }
             uint8_t* sd = smem + args.off_sc + rc.s * args.sc_slot_bytes;
             const int xs = 4 * G * (kt / G);
-            mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * n16) * 4 * G));
-            tma_load_3d(sd, &smap0, xs, y0, e, &sc_full[rc.s], pol);
-            tma_load_3d(sd + 128 * 4 * G, MODE == 0 ? &smap1 : &smap0, xs, y1, e, &sc_full[rc.s], pol);
-            for (int p = 0; p < P; ++p)
-              for (int j = 0; j < n16; j += kTcBoxRows)
-                tma_load_2d(sd + (256 + p * n16 + j) * 4 * G, &tsmap, xs, p * args.pairs + pos0 + j, &sc_full[rc.s]);
+            mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * NC) * 4 * G));
+            tma_load_3d(sd, &smap0, xs, y0, e, &sc_full[rc.s], pol);  // MODE 1: both tiles' 256 rows
+            if (MODE == 0) tma_load_3d(sd + 128 * 4 * G, &smap1, xs, y0, e, &sc_full[rc.s], pol);
+            tma_load_3d_nohint(sd + 256 * 4 * G, &tsmap, xs, pos0, 0, &sc_full[rc.s]);  // [term][n_chunk rows]
             rc.next();
             ++sc_issued;
           }
@@ -424,12 +444,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           }
           mbar_arrive_expect_tx(&full[rs.s], tx);
           uint8_t* dst = smem + rs.s * args.stage_bytes;
-          tma_load_3d(dst, &wmap0, kt * kMxKT, y0, e, &full[rs.s], pol);
-          tma_load_3d(dst + kMxTileBytes, MODE == 0 ? &wmap1 : &wmap0, kt * kMxKT, y1, e, &full[rs.s], pol);
-          uint8_t* bdst = dst + 2 * kMxTileBytes;
-          for (int p = 0; p < P; ++p)
-            for (int j = 0; j < n16; j += kTcBoxRows)
-              tma_load_2d(bdst + (p * n16 + j) * 128, &bmap, kt * kMxKT, p * args.pairs + pos0 + j, &full[rs.s]);
+          tma_load_3d(dst, &wmap0, kt * kMxKT, y0, e, &full[rs.s], pol);  // MODE 1: both 128-row tiles
+          if (MODE == 0) tma_load_3d(dst + kMxTileBytes, &wmap1, kt * kMxKT, y0, e, &full[rs.s], pol);
+          tma_load_3d_nohint(dst + 2 * kMxTileBytes, &bmap, kt * kMxKT, pos0, 0, &full[rs.s]);
           rs.next();
           ++issued;
         }
@@ -462,9 +479,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         const int n16 = (n + 15) & ~15;
-        // summed terms: one MMA of N = tokens per term; stacked: one of N = P x tokens
+        // summed terms: one MMA of N = tokens per term; stacked: one of N = P x
+        // n_chunk over every term's block of token rows
         const int nmma = summed ? P : 1;
-        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, summed ? n16 : P * n16);
+        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, summed ? n16 : P * NC);
         const int b = (int)(un % (uint32_t)NB);
         const uint32_t acc0 = tbase + (uint32_t)(b * 2 * args.acc_cols), acc1 = acc0 + args.acc_cols;
         if (!mbar_wait(&acc_empty[b], ((un / NB) & 1) ^ 1)) {
@@ -484,7 +502,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           }
           tc_fence_after();
           // this stage's operands: weight tiles at 0 and 16 KB, token rows at 32 KB
-          // (term p's n16 rows p * n16 * 128 bytes further); a k-block is 32 bytes
+          // (term p's block p * n_chunk * 128 bytes further); a k-block is 32 bytes
           const uint64_t da0 = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
           const uint64_t da1 = da0 + (kMxTileBytes >> 4), db = da0 + (2 * kMxTileBytes >> 4);
           const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
@@ -496,7 +514,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             const uint32_t sel = (uint32_t)kb << 30;
             const uint64_t ko = (uint64_t)(2 * kb);
             for (int p = 0; p < nmma; ++p) {
-              const uint64_t bd = db + ko + (uint64_t)((p * n16 * 128) >> 4);
+              const uint64_t bd = db + ko + (uint64_t)((p * NC * 128) >> 4);
               const uint32_t sfb = (sfb0 + 4 * p) | sel;
               const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
               umma_mx(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
@@ -527,7 +545,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x) {
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
-      const int n16 = (n + 15) & ~15;
       bool ok = true;
       for (int g = 0; g < nkt / G; ++g) {
         // the stage's E8M0 rows: from the scale ring (TMA) or straight from memory
@@ -558,8 +575,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             for (int j = 0; j < G; ++j) a[8 * j + 4 * m + c] = w[j];
           }
         // token scales, 4 columns at a time: stacked, column c holds N index
-        // 32 c + lane (term nn / n16, token nn mod n16); summed, block p of 4
-        // columns holds term p, column c of it token 32 c + lane
+        // 32 c + lane (term nn / n_chunk, token nn mod n_chunk); summed, block p
+        // of 4 columns holds term p, column c of it token 32 c + lane
         auto load_tokens = [&](int q4) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -569,14 +586,14 @@ __global__ void __launch_bounds__(kMxThreads, 1)
               t = 32 * c + lane;
             } else {
               const int nn = 32 * c + lane;
-              p = nn / n16;
-              t = nn - p * n16;
+              p = nn / NC;
+              t = nn - p * NC;
             }
             uint32_t w[G];
 #pragma unroll
             for (int j = 0; j < G; ++j) w[j] = 0;
             if (p < P && t < n) {
-              if (ss != nullptr) load_words_smem<G>(ss + (256 + p * n16 + t) * 4 * G, w);
+              if (ss != nullptr) load_words_smem<G>(ss + (256 + p * NC + t) * 4 * G, w);
               else load_words<G>(args.b_scale + ((int64_t)p * args.pairs + pos0 + t) * sr + 4 * G * g, w);
             }
 #pragma unroll
@@ -626,7 +643,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     for (int u = blockIdx.x; u < n_units && !__any_sync(0xffffffffu, aborted() ? 1 : 0); u += gridDim.x, ++un) {
       int e, mt, pos0, n;
       decode_unit(u, e, mt, pos0, n);
-      const int n16 = (n + 15) & ~15;
       const int b = (int)(un % (uint32_t)NB);
       const uint32_t accb = tbase + lrow + (uint32_t)(b * 2 * args.acc_cols);
       if (!warp_wait(&acc_full[b], (un / NB) & 1)) {
@@ -641,8 +657,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         for (int j = 0; j < 16; ++j) g[j] = v[j] = 0.f;
         for (int p = 0; p < pe; ++p) {
           uint32_t t0[16], t1[16];
-          tmem_ld16(accb + p * n16 + c0, t0);
-          tmem_ld16(accb + args.acc_cols + p * n16 + c0, t1);
+          tmem_ld16(accb + p * NC + c0, t0);
+          tmem_ld16(accb + args.acc_cols + p * NC + c0, t1);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -652,24 +668,32 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
         if (MODE == 0) {
           // h of row col for 16 tokens, split into E4M3 terms; the 32 lanes of
-          // the warp are one group of 32 h values of a token (the down GEMM's k)
+          // the warp are one group of 32 h values of a token (the down GEMM's
+          // k).  The 16 tokens are independent, so each step runs for all of
+          // them before the next (their reductions and conversions overlap);
+          // tokens past the chunk are computed and not stored.
           const int col = mt * 128 + q * 32 + lane;
           uint8_t* hq = static_cast<uint8_t*>(args.out);
+          float r[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < n) {  // the same for the whole warp
-              float r = silu_clamped_swiglu(g[j], v[j], args.limit);
-              const int64_t pos = pos0 + c0 + j;
-              for (int p = 0; p < args.out_parts; ++p) {
-                const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r)));
-                const int s = e8m0_of_amax(amax);
-                const uint32_t code = e4m3_rn(r * e8m0_inv(s));
-                const int64_t row = (int64_t)p * args.pairs + pos;
+          for (int j = 0; j < 16; ++j) r[j] = silu_clamped_swiglu(g[j], v[j], args.limit);
+          const int nj = n - c0;  // tokens of this 16-chunk that exist (warp-uniform)
+          for (int p = 0; p < args.out_parts; ++p) {
+            uint32_t amax[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) amax[j] = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[j])));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int s = e8m0_of_amax(amax[j]);
+              const uint32_t code = e4m3_rn(r[j] * e8m0_inv(s));
+              if (j < nj) {
+                const int64_t row = (int64_t)p * args.pairs + pos0 + c0 + j;
                 hq[row * args.rows + col] = (uint8_t)code;
                 if (lane == 0) args.out_scale[row * (args.rows / 32) + col / 32] = (uint8_t)s;
-                r -= e4m3_val(code) * e8m0_val(s);
               }
+              r[j] -= e4m3_val(code) * e8m0_val(s);
             }
+          }
         } else {
           float* out = static_cast<float*>(args.out);
           const int col = mt * 256 + q * 32 + lane;
@@ -715,7 +739,12 @@ __global__ void gather_split_kernel(const uint4* __restrict__ x, const int32_t* 
     if (ok) {
       pos = i / h8;
       c8 = (int)(i - pos * h8);
-      const int64_t t = perm[pos] / top_k;
+      int64_t pid = perm[pos];
+      if (kDebug && (pid < 0 || pid >= pairs)) {
+        set_error(kErrBadIndex);
+        pid = 0;
+      }
+      const int64_t t = pid / top_k;
       const uint4 w = x[t * h8 + c8];
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll

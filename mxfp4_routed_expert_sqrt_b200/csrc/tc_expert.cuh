@@ -333,6 +333,16 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   if (grouped)
     for (int i = tid; i <= E; i += blockDim.x) s_off[i] = args.offsets[i];
   __syncthreads();
+  if (kDebug && grouped) {  // offsets must not decrease (the pair count bounds them above)
+    bool bad = false;
+    for (int i = tid; i < E; i += blockDim.x) bad |= s_off[i] > s_off[i + 1];
+    if (tid == 0) bad |= s_off[0] != 0;
+    if (__syncthreads_or(bad ? 1 : 0)) {
+      if (tid == 0) set_error(kErrBadOffsets);
+      for (int i = tid; i <= E; i += blockDim.x) s_off[i] = 0;  // no units
+      __syncthreads();
+    }
+  }
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < E; base += 32) {
@@ -620,7 +630,6 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
-        const int n16 = (n + 15) & ~15;  // rows past the chunk are loaded but never stored
         bool ok = true;
         for (int st = 0; st < nst; ++st) {
           if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
@@ -628,13 +637,14 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&b_full[rs.s], (uint32_t)(kTcKG * n16 * 128));
+          // one box of n_chunk token rows per k-block (rows past the unit's
+          // tokens are loaded but never stored)
+          mbar_arrive_expect_tx(&b_full[rs.s], (uint32_t)(kTcKG * NC * 128));
           uint8_t* dst = s_b + rs.s * bst;
 #pragma unroll
           for (int g = 0; g < kTcKG; ++g) {
             const int col = (st * kTcStageK + g * kTcKB) % args.b_cols;
-            for (int j = 0; j < n16; j += kTcBoxRows)
-              tma_load_2d(dst + g * atom + j * 128, &bmap, col, pos0 + j, &b_full[rs.s]);
+            tma_load_2d(dst + g * atom, &bmap, col, pos0, &b_full[rs.s]);
           }
           rs.next();
           ++issued;
@@ -786,7 +796,12 @@ __global__ void gather_f16_kernel(const uint4* __restrict__ x, const int32_t* __
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / h8;
     const int c = (int)(i - row * h8);
-    const uint4 v = x[(int64_t)(perm[row] / K) * h8 + c];
+    int64_t pid = perm[row];
+    if (kDebug && (pid < 0 || pid >= rows)) {
+      set_error(kErrBadIndex);
+      pid = 0;
+    }
+    const uint4 v = x[(int64_t)(pid / K) * h8 + c];
     const uint4 o = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
     inf |= f16x2_has_inf(o.x) | f16x2_has_inf(o.y) | f16x2_has_inf(o.z) | f16x2_has_inf(o.w);
     out[i] = o;

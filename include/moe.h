@@ -98,6 +98,11 @@ const char* moe_status_string(moe_status status);
  *          bytes span more than 36 octaves and flushed its lowest groups;
  *   0x303  moe_expert_gemm's dequantising path met an activation beyond the
  *          f16 range (|x| > 65504); that call's output is undefined;
+ *   0x304  moe_expert_gemm's dequantising path produced an h (between the
+ *          GEMMs, f16) whose 32 rows of a unit all fell below f16's normal
+ *          range (2^-14): those outputs kept only f16-subnormal precision;
+ *   0x501  debug build: a pair index (perm / inv) outside [0, T * top_k);
+ *   0x502  debug build: group offsets not non-decreasing from 0;
  *   0x401  moe_selftest_wait. */
 int32_t moe_device_error(void);
 
@@ -218,9 +223,11 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *    x goes in as f16: exact for |x| in [2^-17, 65504], f16 subnormal
  *    precision below (absolute error at most 2^-25); a value beyond 65504
  *    is not representable and the call records device error 0x303 (its
- *    output is undefined).  h between the GEMMs is f16; f16 x f16 MMAs with
- *    fp32 sums.  Workspace: x in expert order as f16 [T*top_k][hidden], then
- *    h in f16 [T*top_k][inter].
+ *    output is undefined).  h between the GEMMs is f16 (11 significant bits
+ *    down to 2^-14, subnormal below; a unit whose h all lies below 2^-14
+ *    records device error 0x304); f16 x f16 MMAs with fp32 sums.
+ *    Workspace: x in expert order as f16 [T*top_k][hidden], then h in f16
+ *    [T*top_k][inter].
  * Shapes: inter a multiple of 128, hidden a multiple of 256 (the row tiles of
  * the two GEMMs), besides the moe_dims limits; other shapes return
  * MOE_ERR_UNSUPPORTED before anything is enqueued.

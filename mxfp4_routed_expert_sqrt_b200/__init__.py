@@ -144,6 +144,7 @@ DEVICE_ERR_BAD_EXPERT = 0x201
 DEVICE_ERR_WAIT_TC = 0x301
 DEVICE_ERR_SPAN_FLUSH = 0x302
 DEVICE_ERR_F16_RANGE = 0x303
+DEVICE_ERR_F16_SMALL = 0x304
 DEVICE_ERR_WAIT_SELFTEST = 0x401
 DEVICE_ERR_BAD_INDEX = 0x501     # debug build only
 DEVICE_ERR_BAD_OFFSETS = 0x502   # debug build only

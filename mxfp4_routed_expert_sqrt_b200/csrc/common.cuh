@@ -19,6 +19,7 @@ enum : int32_t {
   kErrWaitTc = 0x301,       // tensor-core kernel gave up waiting on an mbarrier
   kErrSpanFlush = 0x302,    // a weight row's E8M0 bytes span > 36 octaves: the lowest groups were flushed
   kErrF16Range = 0x303,     // an activation beyond the f16 range reached the dequantising expert path
+  kErrF16Small = 0x304,     // dequantising path: every h of a unit's 32 rows fell below f16's normal range
   kErrWaitSelftest = 0x401, // moe_selftest_wait: its wait ran out, as it should
   kErrBadIndex = 0x501,     // debug build: a pair index (perm / inv) outside [0, T * top_k)
   kErrBadOffsets = 0x502,   // debug build: group offsets not non-decreasing from 0 to T * top_k

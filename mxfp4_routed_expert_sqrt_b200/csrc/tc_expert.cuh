@@ -732,6 +732,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
         s0 = pow2_f32(s_crow[un % kCrowRing][0][r]);
         s1 = pow2_f32(s_crow[un % kCrowRing][1][r]);
       }
+      float hmax = 0.f;  // MXFP4 gate/up: the largest |h| of this warp's rows in the unit
       for (int c0 = 16 * half; c0 < n; c0 += 16 * (EPI / 4)) {
         uint32_t g[16], h[16];
         tmem_ld16(tbase + lrow + c0, g);
@@ -747,6 +748,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
               const int64_t o = (int64_t)(pos0 + c0 + j);
               if (AF == kAMxfp4) {
                 static_cast<__half*>(args.out)[o * args.rows + col] = __float2half_rn(hv);
+                hmax = fmaxf(hmax, fabsf(hv));
               } else {
                 const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out) + o * 2 * args.rows;
@@ -764,6 +766,12 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
               out[(int64_t)(pos0 + c0 + j) * args.rows + col + 128] = __uint_as_float(h[j]) * s1;
             }
         }
+      }
+      if (MODE == 0 && AF == kAMxfp4) {
+        // h travels to the down GEMM in f16: if none of it reaches f16's
+        // normal range (2^-14), it kept only subnormal precision -- flagged
+        const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(hmax)));
+        if (lane == 0 && m > 0.f && m < 6.103515625e-05f) set_error(kErrF16Small);
       }
       tc_fence_before();
       __syncwarp();

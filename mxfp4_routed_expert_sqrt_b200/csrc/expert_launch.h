@@ -53,7 +53,6 @@ struct MxLayout {
 // unit's epilogue runs (measured on one B200: the batch-64 expert call 1088 ->
 // 1003 us).
 constexpr int kMxDecodeBufs = 2;  // accumulator sets of the stacked (decode) layout
-constexpr int kMxPrefetchKt = 0;  // K-tiles of weights the loader prefetches into L2 ahead
 inline MxLayout mx_layout(int T, int K, int E) {
   const int64_t avg = ((int64_t)T * K + E - 1) / E;
   if (avg <= 8) return {32, 0, kMxDecodeBufs};
@@ -108,7 +107,6 @@ inline bool mx_launch_args(const moe_dims& dims, int T, const moe_mxfp4_proj& ga
   g.n_chunk = lay.chunk;
   g.term_acc = lay.term_acc;
   g.max_bufs = lay.max_bufs;
-  g.prefetch = kMxPrefetchKt;
   g.out = L.hq;
   g.out_scale = L.hs;
   g.out_parts = kHTerms;

@@ -176,30 +176,34 @@ moe_status launch_tc(const CUtensorMap& bmap, const TcArgs& a, cudaStream_t s) {
 }
 
 // E2M1 plane of an MXFP4 weight array viewed by the block-scaled expert
-// kernel's loader: {columns (codes), rows, experts}, boxes of 128 codes x
-// box_rows rows (128: one tile; 256: both tiles of a down unit) widened to the
-// f8f6f4 shared-memory layout (16U4_ALIGN16B), 128-byte swizzle.
+// kernel's loader as {codes of a K-tile (128), rows, K-tiles, experts}: boxes of
+// 128 codes x box_rows rows (128: one tile; 256: both tiles of a down unit) x
+// kps K-tiles, widened to the f8f6f4 shared-memory layout (16U4_ALIGN16B),
+// 128-byte swizzle; in shared memory [K-tile][row][128 B].
 bool make_mx_weight_map(CUtensorMap* map, const uint8_t* base, const MxArgs& a, int box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr || base == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)a.cols, (cuuint64_t)a.rows, (cuuint64_t)a.E};
-  cuuint64_t strides[2] = {(cuuint64_t)a.cols / 2, (cuuint64_t)a.expert_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)kMxKT, (cuuint32_t)box_rows, 1}, estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+  cuuint64_t dims[4] = {(cuuint64_t)kMxKT, (cuuint64_t)a.rows, (cuuint64_t)(a.cols / kMxKT), (cuuint64_t)a.E};
+  cuuint64_t strides[3] = {(cuuint64_t)a.cols / 2, (cuuint64_t)kMxKT / 2, (cuuint64_t)a.expert_bytes};
+  cuuint32_t box[4] = {(cuuint32_t)kMxKT, (cuuint32_t)box_rows, (cuuint32_t)a.kps, 1}, estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E4M3 token terms [parts][pairs][cols] bytes viewed as {cols, pairs, parts}
-// with one {128, n_chunk, parts} box per stage (every term's rows of a unit in
-// one copy), 128-byte swizzle.
-bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t pairs, int parts, int64_t cols, int n_chunk) {
+// E4M3 token terms [parts][pairs][cols] bytes viewed as {bytes of a K-tile
+// (128), pairs, parts, K-tiles} with one {128, n_chunk, parts, kps} box per
+// stage (every term's rows of a unit for the stage's K-tiles in one copy),
+// 128-byte swizzle; in shared memory [K-tile][term][row][128 B].
+bool make_term_map(CUtensorMap* map, const uint8_t* base, int64_t pairs, int parts, int64_t cols, int n_chunk,
+                   int kps) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)pairs, (cuuint64_t)parts};
-  cuuint64_t strides[2] = {(cuuint64_t)cols, (cuuint64_t)(cols * pairs)};
-  cuuint32_t box[3] = {(cuuint32_t)kMxKT, (cuuint32_t)n_chunk, (cuuint32_t)parts}, estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+  cuuint64_t dims[4] = {(cuuint64_t)kMxKT, (cuuint64_t)pairs, (cuuint64_t)parts, (cuuint64_t)(cols / kMxKT)};
+  cuuint64_t strides[3] = {(cuuint64_t)cols, (cuuint64_t)(cols * pairs), (cuuint64_t)kMxKT};
+  cuuint32_t box[4] = {(cuuint32_t)kMxKT, (cuuint32_t)n_chunk, (cuuint32_t)parts, (cuuint32_t)kps};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -510,8 +514,8 @@ moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t
                            L.xq, L.xs);
   if (st != MOE_OK) return st;
   CUtensorMap xmap, hmap;
-  if (!make_term_map(&xmap, L.xq, L.pairs, kXTerms, H, L.g.n_chunk) ||
-      !make_term_map(&hmap, L.hq, L.pairs, kHTerms, I, L.d.n_chunk))
+  if (!make_term_map(&xmap, L.xq, L.pairs, kXTerms, H, L.g.n_chunk, L.g.kps) ||
+      !make_term_map(&hmap, L.hq, L.pairs, kHTerms, I, L.d.n_chunk, L.d.kps))
     return MOE_ERR_CUDA;
   if ((st = launch_mx<0>(xmap, L.g, s)) != MOE_OK) return st;
   return launch_mx<1>(hmap, L.d, s);

@@ -98,7 +98,6 @@ struct MxArgs {
   uint8_t* out_scale;    // MODE 0: E8M0 of h [out_parts][pairs][rows / 32]
   int out_parts;
   float limit;
-  int prefetch;          // K-tiles of weights prefetched into L2 ahead of the loads (0: none)
   // filled in by mx_plan()
   int g;             // K-tiles per scale stage
   int acc_cols;      // TMEM columns per accumulator
@@ -107,7 +106,8 @@ struct MxArgs {
   int sf_kt;         // TMEM columns per K-tile in a scale stage (8 weight + tok_cols)
   int sf_stages;     // scale stages in TMEM
   int stages;        // shared-memory stages
-  int stage_bytes;   // weights + token rows of one stage
+  int kps;           // K-tiles per shared-memory stage (1 or 2)
+  int stage_bytes;   // weights + token rows of one stage (kps K-tiles)
   int tma_scales;    // 1: E8M0 rows arrive by TMA in a shared-memory scale ring
   int sc_slot_bytes; // one scale-ring slot: [2 x 128 weight rows + parts x n_chunk token rows][4 G]
   int off_sc;        // scale ring
@@ -144,13 +144,17 @@ inline bool mx_plan(MxArgs& a, int mode) {
   if (a.g == 0) return false;
   a.sf_stages = (kTcTmemCols - a.acc_bufs * 2 * a.acc_cols) / (a.sf_kt * a.g);
   if (a.sf_stages > kMxMaxSfStages) a.sf_stages = kMxMaxSfStages;
-  a.stage_bytes = 2 * kMxTileBytes + a.parts * nc * 128;
   const int pre = (2 * (a.E + 1) * 4 + 127) / 128 * 128;
   const int budget = kTcSmemMax - 1024;
   // scale rows by TMA: rows of 4 G bytes, a multiple of 16, with row strides
   // (cols / 32 bytes) a multiple of 16; otherwise the scale writers load them
   a.tma_scales = (a.cols / 32) % 16 == 0 && a.g >= 4 ? 1 : 0;
   a.sc_slot_bytes = a.tma_scales ? ((256 + a.parts * nc) * 4 * a.g + 127) / 128 * 128 : 0;
+  // stages of two K-tiles where two of them fit beside two scale slots (half
+  // the stage handshakes and TMA instructions per weight byte), else one
+  const int kt_bytes = 2 * kMxTileBytes + a.parts * nc * 128;  // one K-tile's weights + token rows
+  a.kps = nkt % 2 == 0 && a.g % 2 == 0 && 2 * 2 * kt_bytes + 2 * a.sc_slot_bytes + pre <= budget ? 2 : 1;
+  a.stage_bytes = a.kps * kt_bytes;
   auto weight_stages = [&]() { return (budget - pre - a.sf_stages * a.sc_slot_bytes) / a.stage_bytes; };
   a.stages = weight_stages();
   while (a.tma_scales && a.stages < 4 && a.sf_stages > 2) {  // keep weight stages over scale slots
@@ -177,14 +181,23 @@ __device__ __forceinline__ void tma_load_3d_nohint(void* dst, const CUtensorMap*
       : "memory");
 }
 
-// Box {x, y, z} of a 3-D tensor map into L2 only (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
-               : "memory");
+// Box {x, y, z, w} of a 4-D tensor map into shared memory (no cache hint).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
 }
-// Contiguous bytes into L2 (16-byte aligned address, size a multiple of 16).
-__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+// The same with an L2 cache hint.
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+      "{%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
 }
 
 // Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both
@@ -289,6 +302,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   const int TC = args.tok_cols;
   const uint32_t sf_base = NB * 2 * args.acc_cols;
   const int sf_cols = args.sf_kt * G;
+  const int KPS = args.kps;  // K-tiles per shared-memory stage
 
   // ---- unit table: units(e) = MT * ceil(n_e / NC), exclusive prefix ----------
   griddep_wait();  // the offsets and token terms come from earlier kernels of the stream
@@ -381,30 +395,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (lane == 0) {
       TcRing rs(args.stages);
       const uint64_t pol = policy_evict_first();
-      // L2 prefetch cursor, args.prefetch K-tiles ahead of the loads (across
-      // units): more HBM bytes in flight than the shared-memory ring holds.
-      // At a unit's first prefetch its E8M0 rows (contiguous per tile) go too.
-      const int64_t plane = (int64_t)args.rows * (args.cols / 2);
-      int pu = blockIdx.x, pkt = 0, pe = 0, pmt = 0, ppos = 0, pn = 0;
-      auto pf_step = [&]() {
-        if (pu >= n_units) return;
-        if (pkt == 0) {
-          decode_unit(pu, pe, pmt, ppos, pn);
-          const int r0 = MODE == 0 ? pmt * 128 : pmt * 256;
-          const uint32_t bytes = (uint32_t)((MODE == 0 ? 128 : 256) * sr);
-          l2_prefetch(args.w0 + (int64_t)pe * args.expert_bytes + plane + (int64_t)r0 * sr, bytes);
-          if (MODE == 0) l2_prefetch(args.w1 + (int64_t)pe * args.expert_bytes + plane + (int64_t)r0 * sr, bytes);
-        }
-        const int y0 = MODE == 0 ? pmt * 128 : pmt * 256;
-        const int y1 = MODE == 0 ? pmt * 128 : pmt * 256 + 128;
-        tma_prefetch_3d(&wmap0, pkt * kMxKT, y0, pe);
-        tma_prefetch_3d(MODE == 0 ? &wmap1 : &wmap0, pkt * kMxKT, y1, pe);
-        if (++pkt == nkt) {
-          pkt = 0;
-          pu += gridDim.x;
-        }
-      };
-      for (int i = 0; i < args.prefetch; ++i) pf_step();
       int issued = 0, sc_issued = 0;
       TcRing rc(args.sf_stages);  // scale-ring slots, one per scale stage
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
@@ -413,12 +403,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         decode_unit(u, e, mt, pos0, n);
         (void)n;
         const int y0 = MODE == 0 ? mt * 128 : mt * 256;
-        // one stage: both weight tiles (MODE 1: one 256-row box) and one box of
-        // every term's n_chunk token rows (rows past the unit's tokens are
-        // loaded but never stored)
-        const uint32_t tx = 2 * kMxTileTx + (uint32_t)(P * NC * 128);
+        // one stage = KPS K-tiles: both weight tiles' KPS K-tiles (MODE 0: a
+        // box per projection; MODE 1: one box of 256 rows), then one box of
+        // every term's n_chunk token rows for the KPS K-tiles (rows past the
+        // unit's tokens are loaded but never stored)
+        const uint32_t tx = (uint32_t)KPS * (2 * kMxTileTx + (uint32_t)(P * NC * 128));
         bool ok = true;
-        for (int kt = 0; kt < nkt; ++kt) {
+        for (int kt = 0; kt < nkt; kt += KPS) {
           if (args.tma_scales && kt % G == 0) {
             // the scale stage's E8M0 rows: both weight tiles, then every term's
             // token rows, [row][4 G bytes]
@@ -436,7 +427,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             rc.next();
             ++sc_issued;
           }
-          if (args.prefetch > 0) pf_step();
           if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
             give_up();
             ok = false;
@@ -444,9 +434,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           }
           mbar_arrive_expect_tx(&full[rs.s], tx);
           uint8_t* dst = smem + rs.s * args.stage_bytes;
-          tma_load_3d(dst, &wmap0, kt * kMxKT, y0, e, &full[rs.s], pol);  // MODE 1: both 128-row tiles
-          if (MODE == 0) tma_load_3d(dst + kMxTileBytes, &wmap1, kt * kMxKT, y0, e, &full[rs.s], pol);
-          tma_load_3d_nohint(dst + 2 * kMxTileBytes, &bmap, kt * kMxKT, pos0, 0, &full[rs.s]);
+          // [KPS][rows][128 B] per projection (MODE 1: [KPS][256][128 B])
+          tma_load_4d_hint(dst, &wmap0, 0, y0, kt, e, &full[rs.s], pol);
+          if (MODE == 0) tma_load_4d_hint(dst + KPS * kMxTileBytes, &wmap1, 0, y0, kt, e, &full[rs.s], pol);
+          tma_load_4d(dst + 2 * KPS * kMxTileBytes, &bmap, 0, pos0, 0, kt, &full[rs.s]);  // [KPS][P][NC][128 B]
           rs.next();
           ++issued;
         }
@@ -490,44 +481,54 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           break;
         }
         tc_fence_after();
-        for (int kt = 0; kt < nkt; ++kt) {
-          const int j = kt % G;
-          if (j == 0 && !mbar_wait(&sf_full[rf.s], rf.ph)) {
-            ok = false;
-            break;
-          }
+        for (int kt0 = 0; kt0 < nkt && ok; kt0 += KPS) {
           if (!mbar_wait(&full[rs.s], rs.ph)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // this stage's operands: weight tiles at 0 and 16 KB, token rows at 32 KB
-          // (term p's block p * n_chunk * 128 bytes further); a k-block is 32 bytes
-          const uint64_t da0 = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
-          const uint64_t da1 = da0 + (kMxTileBytes >> 4), db = da0 + (2 * kMxTileBytes >> 4);
-          const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
-          const uint32_t sfa0 = sfc + 8 * j, sfa1 = sfa0 + 4, sfb0 = sfc + 8 * G + TC * j;
-          const uint32_t first = kt > 0 ? 1u : 0u;
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
-            const uint32_t sel = (uint32_t)kb << 30;
-            const uint64_t ko = (uint64_t)(2 * kb);
-            for (int p = 0; p < nmma; ++p) {
-              const uint64_t bd = db + ko + (uint64_t)((p * NC * 128) >> 4);
-              const uint32_t sfb = (sfb0 + 4 * p) | sel;
-              const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
-              umma_mx(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
-              umma_mx(acc1, da1 + ko, bd, id, acc, sfa1 | sel, sfb);
+          // this stage's operands: MODE 0 gate K-tiles at 0, up K-tiles at KPS x
+          // 16 KB; MODE 1 K-tile kk's 256 rows at kk x 32 KB (tile 1 16 KB in);
+          // token rows at 2 KPS x 16 KB, [kk][term][n_chunk][128 B]; a k-block
+          // is 32 bytes
+          const uint64_t ds = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
+          for (int kk = 0; kk < KPS; ++kk) {
+            const int kt = kt0 + kk, j = kt % G;
+            if (j == 0) {
+              if (!mbar_wait(&sf_full[rf.s], rf.ph)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();  // the scale writers' tcgen05.st before this stage's MMAs
             }
+            const uint64_t da0 = ds + (uint64_t)((MODE == 0 ? kk * kMxTileBytes : kk * 2 * kMxTileBytes) >> 4);
+            const uint64_t da1 = MODE == 0 ? da0 + (uint64_t)((KPS * kMxTileBytes) >> 4) : da0 + (kMxTileBytes >> 4);
+            const uint64_t db = ds + (uint64_t)((2 * KPS * kMxTileBytes + kk * P * NC * 128) >> 4);
+            const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
+            const uint32_t sfa0 = sfc + 8 * j, sfa1 = sfa0 + 4, sfb0 = sfc + 8 * G + TC * j;
+            const uint32_t first = kt > 0 ? 1u : 0u;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
+              const uint32_t sel = (uint32_t)kb << 30;
+              const uint64_t ko = (uint64_t)(2 * kb);
+              for (int p = 0; p < nmma; ++p) {
+                const uint64_t bd = db + ko + (uint64_t)((p * NC * 128) >> 4);
+                const uint32_t sfb = (sfb0 + 4 * p) | sel;
+                const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
+                umma_mx(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
+                umma_mx(acc1, da1 + ko, bd, id, acc, sfa1 | sel, sfb);
+              }
+            }
+            if (j == G - 1) {
+              umma_commit(&sf_empty[rf.s]);
+              rf.next();
+            }
+            if (kt == nkt - 1) umma_commit(&acc_full[b]);
           }
+          if (!ok) break;
           umma_commit(&empty[rs.s]);
           rs.next();
-          if (j == G - 1) {
-            umma_commit(&sf_empty[rf.s]);
-            rf.next();
-          }
-          if (kt == nkt - 1) umma_commit(&acc_full[b]);
         }
       }
       if (!ok) give_up();

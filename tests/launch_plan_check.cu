@@ -47,7 +47,12 @@ static void check_mx_plan(const MxArgs& a, int mode, const char* name, int T) {
   CHECK(a.sf_stages >= 2 && a.sf_stages <= kMxMaxSfStages && a.stages >= 2, "%s T=%d rings", name, T);
   CHECK((a.cols / kMxKT) % a.g == 0, "%s T=%d G", name, T);
   CHECK(a.stage_bytes % 1024 == 0, "%s T=%d stage", name, T);
-  CHECK(a.stage_bytes >= 2 * kMxTileBytes + a.parts * a.n_chunk * 128, "%s T=%d stage size", name, T);
+  // a stage holds kps K-tiles of both weight tiles and every term's n_chunk
+  // token rows; two-K-tile stages need an even K-tile count and scale stage
+  CHECK(a.kps == 1 || a.kps == 2, "%s T=%d kps", name, T);
+  CHECK(a.stage_bytes == a.kps * (2 * kMxTileBytes + a.parts * a.n_chunk * 128), "%s T=%d stage size", name, T);
+  CHECK((a.cols / kMxKT) % a.kps == 0 && a.g % a.kps == 0, "%s T=%d kps divides", name, T);
+  CHECK(a.n_chunk <= 256 && a.kps * a.parts <= 256, "%s T=%d box dims", name, T);
   // shared memory: weight stages, then the scale ring (TMA-fed E8M0 rows),
   // then the unit prefix and offsets copy
   CHECK(a.off_sc == a.stages * a.stage_bytes, "%s T=%d scale ring offset", name, T);

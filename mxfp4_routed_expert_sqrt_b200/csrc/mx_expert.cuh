@@ -52,7 +52,8 @@
 //              tcgen05.st them in the layout the MMA reads (below), every
 //              quadrant holding a full copy;
 //   warp 8     loader (one thread): TMA boxes of weights and token terms;
-//   warp 9     TMEM owner and MMA issuer (one thread).
+//   warp 9     TMEM owner and MMA issuer (the whole warp runs the loop, an
+//              elected lane issues each MMA and commit).
 // TMEM (512 columns): acc_bufs accumulator sets (set b: acc0 at 2 b acc,
 // acc1 at 2 b acc + acc), then the scale ring.  With two sets the epilogue of
 // one unit overlaps the MMAs of the next.  A scale stage holds, for K-tile j
@@ -206,12 +207,17 @@ __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N) {
   return (5u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 
-// D[tmem] (+)= (A[smem] * SFA) (B[smem] * SFB)^T, scales from TMEM.
-__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
+// D[tmem] (+)= (A[smem] * SFA) (B[smem] * SFB)^T, scales from TMEM.  Called
+// by all 32 lanes of a converged warp with the same operands; one lane, chosen
+// by elect.sync, issues the MMA.  Issuing from a whole warp lets the operands
+// stay warp-uniform: a lone thread in a lane-0 branch issues one of these
+// every ~80 cycles whatever N is, a warp with an elected lane every ~45
+// (N <= 64; measured with the loop shape below on a B200).
+__device__ __forceinline__ void umma_mx_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
@@ -456,87 +462,85 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------ MMA issuer ----------------------------------
-    if (lane == 0) {
-      TcRing rs(args.stages), rf(args.sf_stages);
-      uint32_t un = 0;
-      bool ok = true;
-      // One thread issues every MMA, so the arithmetic between two MMAs is a
-      // dependent chain that nothing hides: descriptors are built once and
-      // advanced by adding byte offsets / 16 to their 14-bit address field
-      // (every operand lies below 256 KB, so the field never carries into the
-      // constant upper bits).
-      const uint64_t d_smem = sdesc_sw128(smem_u32(smem));
-      for (int u = blockIdx.x; u < n_units && ok && !aborted(); u += gridDim.x, ++un) {
-        int e, mt, pos0, n;
-        decode_unit(u, e, mt, pos0, n);
-        const int n16 = (n + 15) & ~15;
-        // summed terms: one MMA of N = tokens per term; stacked: one of N = P x
-        // n_chunk over every term's block of token rows
-        const int nmma = summed ? P : 1;
-        const uint32_t idesc = idesc_mx_e2m1_e4m3(128, summed ? n16 : P * NC);
-        const int b = (int)(un % (uint32_t)NB);
-        const uint32_t acc0 = tbase + (uint32_t)(b * 2 * args.acc_cols), acc1 = acc0 + args.acc_cols;
-        if (!mbar_wait(&acc_empty[b], ((un / NB) & 1) ^ 1)) {
-          give_up();
+    // The whole warp runs the loop (every wait's outcome is agreed with
+    // __all_sync, so the warp stays converged); an elected lane issues each
+    // MMA and commit.  Descriptors are built once and advanced by adding byte
+    // offsets / 16 to their 14-bit address field (every operand lies below
+    // 256 KB, so the field never carries into the constant upper bits).
+    TcRing rs(args.stages), rf(args.sf_stages);
+    uint32_t un = 0;
+    bool ok = true;
+    const uint64_t d_smem = sdesc_sw128(smem_u32(smem));
+    auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
+    for (int u = blockIdx.x; u < n_units && ok && !warp_aborted(); u += gridDim.x, ++un) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      // summed terms: one MMA of N = tokens per term; stacked: one of N = P x
+      // n_chunk over every term's block of token rows
+      const int nmma = summed ? P : 1;
+      const uint32_t idesc = idesc_mx_e2m1_e4m3(128, summed ? n16 : P * NC);
+      const int b = (int)(un % (uint32_t)NB);
+      const uint32_t acc0 = tbase + (uint32_t)(b * 2 * args.acc_cols), acc1 = acc0 + args.acc_cols;
+      if (!warp_wait(&acc_empty[b], ((un / NB) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int kt0 = 0; kt0 < nkt && ok; kt0 += KPS) {
+        if (!warp_wait(&full[rs.s], rs.ph)) {
+          ok = false;
           break;
         }
         tc_fence_after();
-        for (int kt0 = 0; kt0 < nkt && ok; kt0 += KPS) {
-          if (!mbar_wait(&full[rs.s], rs.ph)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // this stage's operands: MODE 0 gate K-tiles at 0, up K-tiles at KPS x
-          // 16 KB; MODE 1 K-tile kk's 256 rows at kk x 32 KB (tile 1 16 KB in);
-          // token rows at 2 KPS x 16 KB, [kk][term][n_chunk][128 B]; a k-block
-          // is 32 bytes
-          const uint64_t ds = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
-          for (int kk = 0; kk < KPS; ++kk) {
-            const int kt = kt0 + kk, j = kt % G;
-            if (j == 0) {
-              if (!mbar_wait(&sf_full[rf.s], rf.ph)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();  // the scale writers' tcgen05.st before this stage's MMAs
+        // this stage's operands: MODE 0 gate K-tiles at 0, up K-tiles at KPS x
+        // 16 KB; MODE 1 K-tile kk's 256 rows at kk x 32 KB (tile 1 16 KB in);
+        // token rows at 2 KPS x 16 KB, [kk][term][n_chunk][128 B]; a k-block
+        // is 32 bytes
+        const uint64_t ds = d_smem + (uint64_t)((rs.s * args.stage_bytes) >> 4);
+        for (int kk = 0; kk < KPS; ++kk) {
+          const int kt = kt0 + kk, j = kt % G;
+          if (j == 0) {
+            if (!warp_wait(&sf_full[rf.s], rf.ph)) {
+              ok = false;
+              break;
             }
-            const uint64_t da0 = ds + (uint64_t)((MODE == 0 ? kk * kMxTileBytes : kk * 2 * kMxTileBytes) >> 4);
-            const uint64_t da1 = MODE == 0 ? da0 + (uint64_t)((KPS * kMxTileBytes) >> 4) : da0 + (kMxTileBytes >> 4);
-            const uint64_t db = ds + (uint64_t)((2 * KPS * kMxTileBytes + kk * P * NC * 128) >> 4);
-            const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
-            const uint32_t sfa0 = sfc + 8 * j, sfa1 = sfa0 + 4, sfb0 = sfc + 8 * G + TC * j;
-            const uint32_t first = kt > 0 ? 1u : 0u;
+            tc_fence_after();  // the scale writers' tcgen05.st before this stage's MMAs
+          }
+          const uint64_t da0 = ds + (uint64_t)((MODE == 0 ? kk * kMxTileBytes : kk * 2 * kMxTileBytes) >> 4);
+          const uint64_t da1 = MODE == 0 ? da0 + (uint64_t)((KPS * kMxTileBytes) >> 4) : da0 + (kMxTileBytes >> 4);
+          const uint64_t db = ds + (uint64_t)((2 * KPS * kMxTileBytes + kk * P * NC * 128) >> 4);
+          const uint32_t sfc = tbase + sf_base + rf.s * sf_cols;
+          const uint32_t sfa0 = sfc + 8 * j, sfa1 = sfa0 + 4, sfb0 = sfc + 8 * G + TC * j;
+          const uint32_t first = kt > 0 ? 1u : 0u;
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
-              const uint32_t sel = (uint32_t)kb << 30;
-              const uint64_t ko = (uint64_t)(2 * kb);
-              for (int p = 0; p < nmma; ++p) {
-                const uint64_t bd = db + ko + (uint64_t)((p * NC * 128) >> 4);
-                const uint32_t sfb = (sfb0 + 4 * p) | sel;
-                const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
-                umma_mx(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
-                umma_mx(acc1, da1 + ko, bd, id, acc, sfa1 | sel, sfb);
-              }
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t id = idesc | ((uint32_t)kb << 29) | ((uint32_t)kb << 4);
+            const uint32_t sel = (uint32_t)kb << 30;
+            const uint64_t ko = (uint64_t)(2 * kb);
+            for (int p = 0; p < nmma; ++p) {
+              const uint64_t bd = db + ko + (uint64_t)((p * NC * 128) >> 4);
+              const uint32_t sfb = (sfb0 + 4 * p) | sel;
+              const uint32_t acc = (kb > 0 || p > 0) ? 1u : first;
+              umma_mx_warp(acc0, da0 + ko, bd, id, acc, sfa0 | sel, sfb);
+              umma_mx_warp(acc1, da1 + ko, bd, id, acc, sfa1 | sel, sfb);
             }
-            if (j == G - 1) {
-              umma_commit(&sf_empty[rf.s]);
-              rf.next();
-            }
-            if (kt == nkt - 1) umma_commit(&acc_full[b]);
           }
-          if (!ok) break;
-          umma_commit(&empty[rs.s]);
-          rs.next();
+          if (j == G - 1) {
+            umma_commit_warp(&sf_empty[rf.s]);
+            rf.next();
+          }
+          if (kt == nkt - 1) umma_commit_warp(&acc_full[b]);
         }
+        if (!ok) break;
+        umma_commit_warp(&empty[rs.s]);
+        rs.next();
       }
-      if (!ok) give_up();
-      // every MMA of this thread done before TMEM is released
-      umma_commit(&mma_done);
-      if (!mbar_wait(&mma_done, 0)) set_error(kErrWaitTc);
     }
-    __syncwarp();
+    if (!ok && lane == 0) give_up();
+    // every MMA of this warp done before TMEM is released
+    umma_commit_warp(&mma_done);
+    if (!warp_wait(&mma_done, 0) && lane == 0) set_error(kErrWaitTc);
   } else if (warp >= 4) {
     // ------------------------------ scale writers --------------------------------
     const int q = warp & 3;

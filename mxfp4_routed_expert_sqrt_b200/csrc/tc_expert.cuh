@@ -48,7 +48,8 @@
 //               Each thread fetches its row's E8M0 bytes for the NEXT unit with
 //               cp.async into a thread-major buffer;
 //   warp 12     token loader: 2-D TMA boxes of 16 token rows x 64 columns;
-//   warp 13     TMEM owner and MMA issuer (one thread);
+//   warp 13     TMEM owner and MMA issuer (the whole warp runs the loop, an
+//               elected lane issues each MMA and commit);
 //   warp 14     weight loader (one thread): 3-D TMA boxes (128 rows x <= 128
 //               bytes per tile, expert index as the third coordinate) into the
 //               weight ring, running ahead across unit boundaries.
@@ -113,19 +114,25 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc]^T
-__device__ __forceinline__ void umma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem desc]^T.  Called by all 32 lanes of a
+// converged warp with the same operands; one lane, chosen by elect.sync,
+// issues.  A lone thread in a lane-0 branch issues an MMA only every ~80
+// cycles whatever its N (its operands are not warp-uniform); a warp with an
+// elected lane every ~45 (measured on a B200).
+__device__ __forceinline__ void umma_tmem_a_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
+// tcgen05.commit from one elected lane of a converged warp.
+__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
+      : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
@@ -659,57 +666,57 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
-      TcRing rs(args.stages);
-      uint32_t un = 0;
-      // descriptors built once, advanced by byte offset / 16 (operands lie
-      // below 256 KB: the 14-bit address field never carries)
-      const uint64_t d_b = sdesc_sw128(smem_u32(s_b));
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x, ++un) {
-        int e, mt, pos0, n;
-        decode_unit(u, e, mt, pos0, n);
-        const int n16 = (n + 15) & ~15;
-        // MXFP4 weights run as f16 x f16, bf16 weights as bf16 x bf16
-        const uint32_t idesc = AF == kAMxfp4 ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
-        if (!mbar_wait(&acc_empty, (un & 1) ^ 1)) {
-          give_up();
+    // The whole warp runs the loop (wait outcomes agreed with __all_sync, so
+    // it stays converged); an elected lane issues each MMA and commit.
+    // Descriptors are built once and advanced by byte offset / 16 (operands
+    // lie below 256 KB: the 14-bit address field never carries).
+    TcRing rs(args.stages);
+    uint32_t un = 0;
+    const uint64_t d_b = sdesc_sw128(smem_u32(s_b));
+    auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && !warp_aborted(); u += gridDim.x, ++un) {
+      int e, mt, pos0, n;
+      decode_unit(u, e, mt, pos0, n);
+      const int n16 = (n + 15) & ~15;
+      // MXFP4 weights run as f16 x f16, bf16 weights as bf16 x bf16
+      const uint32_t idesc = AF == kAMxfp4 ? idesc_f16_f32(128, n16) : idesc_bf16_f32(128, n16);
+      if (!warp_wait(&acc_empty, (un & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int st = 0; st < nst; ++st) {
+        if (!warp_wait(&full[rs.s], rs.ph)) {
+          ok = false;
           break;
         }
         tc_fence_after();
-        bool ok = true;
-        for (int st = 0; st < nst; ++st) {
-          if (!mbar_wait(&full[rs.s], rs.ph)) {
-            give_up();
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t bd0 = d_b + (uint64_t)((rs.s * bst) >> 4);
-          const uint32_t a0 = tbase + a_base + rs.s * kTcStageCols;
-          const uint32_t acc1 = tbase + args.acc_cols;
-          const uint32_t first = st > 0 ? 1u : 0u;
+        const uint64_t bd0 = d_b + (uint64_t)((rs.s * bst) >> 4);
+        const uint32_t a0 = tbase + a_base + rs.s * kTcStageCols;
+        const uint32_t acc1 = tbase + args.acc_cols;
+        const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
-          for (int g = 0; g < kTcKG; ++g) {
-            const uint64_t bdg = bd0 + (uint64_t)((g * atom) >> 4);
+        for (int g = 0; g < kTcKG; ++g) {
+          const uint64_t bdg = bd0 + (uint64_t)((g * atom) >> 4);
 #pragma unroll
-            for (int ks = 0; ks < kTcKB / 16; ++ks) {
-              const uint64_t bd = bdg + (uint64_t)(2 * ks);
-              const uint32_t acc = (g > 0 || ks > 0) ? 1u : first;
-              umma_tmem_a(tbase, a0 + g * 64 + ks * 8, bd, idesc, acc);
-              umma_tmem_a(acc1, a0 + g * 64 + 32 + ks * 8, bd, idesc, acc);
-            }
+          for (int ks = 0; ks < kTcKB / 16; ++ks) {
+            const uint64_t bd = bdg + (uint64_t)(2 * ks);
+            const uint32_t acc = (g > 0 || ks > 0) ? 1u : first;
+            umma_tmem_a_warp(tbase, a0 + g * 64 + ks * 8, bd, idesc, acc);
+            umma_tmem_a_warp(acc1, a0 + g * 64 + 32 + ks * 8, bd, idesc, acc);
           }
-          umma_commit(&empty[rs.s]);
-          if (st == nst - 1) umma_commit(&acc_full);
-          rs.next();
         }
-        if (!ok) break;
+        umma_commit_warp(&empty[rs.s]);
+        if (st == nst - 1) umma_commit_warp(&acc_full);
+        rs.next();
       }
-      // every MMA of this thread done before TMEM is released
-      umma_commit(&mma_done);
-      if (!mbar_wait(&mma_done, 0)) set_error(kErrWaitTc);
+      if (!ok) break;
     }
-    __syncwarp();
+    if (!ok && lane == 0) give_up();
+    // every MMA of this warp done before TMEM is released
+    umma_commit_warp(&mma_done);
+    if (!warp_wait(&mma_done, 0) && lane == 0) set_error(kErrWaitTc);
   } else if (warp < 4 || (EPI == 8 && warp >= 15)) {
     // ------------------------------ epilogue ----------------------------------
     // MODE 0, MXFP4: h = swiglu(gate, up) in f16 [pos][rows]

@@ -237,10 +237,10 @@ bool make_token_scale_map(CUtensorMap* map, const MxArgs& a) {
 }
 
 // One block-scaled expert launch (planned by mx_plan), one CTA per SM.
-template <int MODE, int G>
+template <int MODE, int G, int KPS, bool SUMMED>
 moe_status launch_mx_g(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
   static std::atomic<uint64_t> configured{0};
-  if (!smem_limit_once(configured, mx_expert_kernel<MODE, G>, kTcSmemMax)) return MOE_ERR_CUDA;
+  if (!smem_limit_once(configured, mx_expert_kernel<MODE, G, KPS, SUMMED>, kTcSmemMax)) return MOE_ERR_CUDA;
   CUtensorMap w0, w1, s0, s1, ts;
   const int box_rows = MODE == 0 ? 128 : 256;  // MODE 1: both 128-row tiles of a unit in one box
   if (!make_mx_weight_map(&w0, a.w0, a, box_rows)) return MOE_ERR_CUDA;
@@ -259,17 +259,26 @@ moe_status launch_mx_g(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s)
   } else {  // unused: the scale writers load the E8M0 rows themselves
     s0 = s1 = ts = w0;
   }
-  return launch_k(mx_expert_kernel<MODE, G>, dim3(sm_count()), dim3(kMxThreads), a.smem_bytes, s, bmap, w0, w1, s0,
+  return launch_k(mx_expert_kernel<MODE, G, KPS, SUMMED>, dim3(sm_count()), dim3(kMxThreads), a.smem_bytes, s, bmap, w0, w1, s0,
                   s1, ts, a);
 }
 
 template <int MODE>
 moe_status launch_mx(const CUtensorMap& bmap, const MxArgs& a, cudaStream_t s) {
+  // the plan gives two-K-tile stages only with an even G
+  const bool k2 = a.kps == 2, sum = a.term_acc != 0;
   switch (a.g) {
-    case 8: return launch_mx_g<MODE, 8>(bmap, a, s);
-    case 4: return launch_mx_g<MODE, 4>(bmap, a, s);
-    case 2: return launch_mx_g<MODE, 2>(bmap, a, s);
-    default: return launch_mx_g<MODE, 1>(bmap, a, s);
+    case 8:
+      return k2 ? (sum ? launch_mx_g<MODE, 8, 2, true>(bmap, a, s) : launch_mx_g<MODE, 8, 2, false>(bmap, a, s))
+                : (sum ? launch_mx_g<MODE, 8, 1, true>(bmap, a, s) : launch_mx_g<MODE, 8, 1, false>(bmap, a, s));
+    case 4:
+      return k2 ? (sum ? launch_mx_g<MODE, 4, 2, true>(bmap, a, s) : launch_mx_g<MODE, 4, 2, false>(bmap, a, s))
+                : (sum ? launch_mx_g<MODE, 4, 1, true>(bmap, a, s) : launch_mx_g<MODE, 4, 1, false>(bmap, a, s));
+    case 2:
+      return k2 ? (sum ? launch_mx_g<MODE, 2, 2, true>(bmap, a, s) : launch_mx_g<MODE, 2, 2, false>(bmap, a, s))
+                : (sum ? launch_mx_g<MODE, 2, 1, true>(bmap, a, s) : launch_mx_g<MODE, 2, 1, false>(bmap, a, s));
+    default:
+      return sum ? launch_mx_g<MODE, 1, 1, true>(bmap, a, s) : launch_mx_g<MODE, 1, 1, false>(bmap, a, s);
   }
 }
 

@@ -406,6 +406,39 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const uint64_t pol = policy_evict_first();
       int issued = 0, sc_issued = 0;
       TcRing rc(args.sf_stages);  // scale-ring slots, one per scale stage
+      // The E8M0 rows of a scale stage (both weight tiles, then every term's
+      // token rows, [row][4 G bytes]) run one scale stage ahead of the weights,
+      // across unit boundaries, so the scale writers find them landed.  The
+      // scale cursor (su, sg) is the next scale stage to load.
+      const int ng = nkt / G;
+      int su = blockIdx.x, sg = 0, s_e = 0, s_y0 = 0, s_pos0 = 0;
+      auto scale_unit = [&]() {
+        int mt_, n_;
+        decode_unit(su, s_e, mt_, s_pos0, n_);
+        s_y0 = MODE == 0 ? mt_ * 128 : mt_ * 256;
+      };
+      if (su < n_units) scale_unit();
+      // issue every scale stage up to (u_lim, g_lim) inclusive; false on a
+      // wait that gave up
+      auto scales_upto = [&](int u_lim, int g_lim) {
+        while (su < n_units && (su < u_lim || (su == u_lim && sg <= g_lim))) {
+          if (!mbar_wait(&sc_empty[rc.s], rc.ph ^ 1)) return false;
+          uint8_t* sd = smem + args.off_sc + rc.s * args.sc_slot_bytes;
+          const int xs = 4 * G * sg;
+          mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * NC) * 4 * G));
+          tma_load_3d(sd, &smap0, xs, s_y0, s_e, &sc_full[rc.s], pol);  // MODE 1: both tiles' 256 rows
+          if (MODE == 0) tma_load_3d(sd + 128 * 4 * G, &smap1, xs, s_y0, s_e, &sc_full[rc.s], pol);
+          tma_load_3d_nohint(sd + 256 * 4 * G, &tsmap, xs, s_pos0, 0, &sc_full[rc.s]);  // [term][n_chunk rows]
+          rc.next();
+          ++sc_issued;
+          if (++sg == ng) {
+            sg = 0;
+            su += gridDim.x;
+            if (su < n_units) scale_unit();
+          }
+        }
+        return true;
+      };
       for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
         if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
@@ -420,21 +453,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         bool ok = true;
         for (int kt = 0; kt < nkt; kt += KPS) {
           if (args.tma_scales && kt % G == 0) {
-            // the scale stage's E8M0 rows: both weight tiles, then every term's
-            // token rows, [row][4 G bytes]
-            if (!mbar_wait(&sc_empty[rc.s], rc.ph ^ 1)) {
+            const int g1 = kt / G + 1;  // this scale stage and the next one
+            if (!(g1 < ng ? scales_upto(u, g1) : scales_upto(u + (int)gridDim.x, 0))) {
               give_up();
               ok = false;
               break;
             }
-            uint8_t* sd = smem + args.off_sc + rc.s * args.sc_slot_bytes;
-            const int xs = 4 * G * (kt / G);
-            mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * NC) * 4 * G));
-            tma_load_3d(sd, &smap0, xs, y0, e, &sc_full[rc.s], pol);  // MODE 1: both tiles' 256 rows
-            if (MODE == 0) tma_load_3d(sd + 128 * 4 * G, &smap1, xs, y0, e, &sc_full[rc.s], pol);
-            tma_load_3d_nohint(sd + 256 * 4 * G, &tsmap, xs, pos0, 0, &sc_full[rc.s]);  // [term][n_chunk rows]
-            rc.next();
-            ++sc_issued;
           }
           if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
             give_up();

@@ -201,6 +201,57 @@ __device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Copies issued from a warp that runs the loader loop as a whole: every lane
+// calls with the same operands and only the lane whose `leader` is nonzero
+// (chosen once with elect.sync) issues, which keeps the operands warp-uniform.
+__device__ __forceinline__ uint32_t elect_leader() {
+  uint32_t r;
+  asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_if(uint32_t leader, uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n}\n" ::"r"(
+                   leader),
+               "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y, int z,
+                                               uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%1], [%2, "
+      "{%3, %4, %5}], [%6], %7;\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_nohint_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y,
+                                                      int z, uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%1], [%2, {%3, %4, %5}], "
+      "[%6];\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y, int z,
+                                               int w, uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%1], [%2, {%3, %4, %5, "
+      "%6}], [%7];\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_hint_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y,
+                                                    int z, int w, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%1], [%2, "
+      "{%3, %4, %5, %6}], [%7], %8;\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both
 // K-major, E8M0 scales, fp32 D; scale-factor ids in bits 4-5 (B) and 29-30 (A).
 __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N) {
@@ -401,7 +452,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 
   if (warp == 8) {
     // ------------------------------ loader -------------------------------------
-    if (lane == 0) {
+    // The whole warp runs the loop (wait outcomes agreed with __all_sync); one
+    // elected lane issues every copy and barrier arrival.
+    {
+      const uint32_t leader = elect_leader();
       TcRing rs(args.stages);
       const uint64_t pol = policy_evict_first();
       int issued = 0, sc_issued = 0;
@@ -422,13 +476,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       // wait that gave up
       auto scales_upto = [&](int u_lim, int g_lim) {
         while (su < n_units && (su < u_lim || (su == u_lim && sg <= g_lim))) {
-          if (!mbar_wait(&sc_empty[rc.s], rc.ph ^ 1)) return false;
+          if (!warp_wait(&sc_empty[rc.s], rc.ph ^ 1)) return false;
           uint8_t* sd = smem + args.off_sc + rc.s * args.sc_slot_bytes;
           const int xs = 4 * G * sg;
-          mbar_arrive_expect_tx(&sc_full[rc.s], (uint32_t)((256 + P * NC) * 4 * G));
-          tma_load_3d(sd, &smap0, xs, s_y0, s_e, &sc_full[rc.s], pol);  // MODE 1: both tiles' 256 rows
-          if (MODE == 0) tma_load_3d(sd + 128 * 4 * G, &smap1, xs, s_y0, s_e, &sc_full[rc.s], pol);
-          tma_load_3d_nohint(sd + 256 * 4 * G, &tsmap, xs, s_pos0, 0, &sc_full[rc.s]);  // [term][n_chunk rows]
+          mbar_arrive_expect_tx_if(leader, &sc_full[rc.s], (uint32_t)((256 + P * NC) * 4 * G));
+          tma_load_3d_if(leader, sd, &smap0, xs, s_y0, s_e, &sc_full[rc.s], pol);  // MODE 1: both tiles' 256 rows
+          if (MODE == 0) tma_load_3d_if(leader, sd + 128 * 4 * G, &smap1, xs, s_y0, s_e, &sc_full[rc.s], pol);
+          tma_load_3d_nohint_if(leader, sd + 256 * 4 * G, &tsmap, xs, s_pos0, 0, &sc_full[rc.s]);  // [term][n_chunk rows]
           rc.next();
           ++sc_issued;
           if (++sg == ng) {
@@ -439,7 +493,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
         return true;
       };
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
+      for (int u = blockIdx.x; u < n_units && !warp_aborted(); u += gridDim.x) {
         if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
@@ -455,22 +510,22 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           if (args.tma_scales && kt % G == 0) {
             const int g1 = kt / G + 1;  // this scale stage and the next one
             if (!(g1 < ng ? scales_upto(u, g1) : scales_upto(u + (int)gridDim.x, 0))) {
-              give_up();
+              if (lane == 0) give_up();
               ok = false;
               break;
             }
           }
-          if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
-            give_up();
+          if (!warp_wait(&empty[rs.s], rs.ph ^ 1)) {
+            if (lane == 0) give_up();
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[rs.s], tx);
+          mbar_arrive_expect_tx_if(leader, &full[rs.s], tx);
           uint8_t* dst = smem + rs.s * args.stage_bytes;
           // [KPS][rows][128 B] per projection (MODE 1: [KPS][256][128 B])
-          tma_load_4d_hint(dst, &wmap0, 0, y0, kt, e, &full[rs.s], pol);
-          if (MODE == 0) tma_load_4d_hint(dst + KPS * kMxTileBytes, &wmap1, 0, y0, kt, e, &full[rs.s], pol);
-          tma_load_4d(dst + 2 * KPS * kMxTileBytes, &bmap, 0, pos0, 0, kt, &full[rs.s]);  // [KPS][P][NC][128 B]
+          tma_load_4d_hint_if(leader, dst, &wmap0, 0, y0, kt, e, &full[rs.s], pol);
+          if (MODE == 0) tma_load_4d_hint_if(leader, dst + KPS * kMxTileBytes, &wmap1, 0, y0, kt, e, &full[rs.s], pol);
+          tma_load_4d_if(leader, dst + 2 * KPS * kMxTileBytes, &bmap, 0, pos0, 0, kt, &full[rs.s]);  // [KPS][P][NC][128 B]
           rs.next();
           ++issued;
         }
@@ -479,11 +534,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       // the last fills must have landed before the CTA exits
       for (int i = 0; i < min(issued, rs.n); ++i) {
         const int s = (rs.s - 1 - i + rs.n) % rs.n;
-        if (!mbar_wait(&full[s], s < rs.s ? rs.ph : rs.ph ^ 1)) set_error(kErrWaitTc);
+        if (!warp_wait(&full[s], s < rs.s ? rs.ph : rs.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
       }
       for (int i = 0; i < min(sc_issued, rc.n); ++i) {
         const int s = (rc.s - 1 - i + rc.n) % rc.n;
-        if (!mbar_wait(&sc_full[s], s < rc.s ? rc.ph : rc.ph ^ 1)) set_error(kErrWaitTc);
+        if (!warp_wait(&sc_full[s], s < rc.s ? rc.ph : rc.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
       }
     }
     __syncwarp();

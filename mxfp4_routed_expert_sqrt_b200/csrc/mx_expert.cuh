@@ -37,11 +37,11 @@
 //   MODE 1 (down):    acc0/acc1 = Wd[2 x 128 rows] h^T over K = inter; fp32 out
 // Swap-AB: weight rows are the MMA's M = 128, token terms its N.
 //
-// Pipeline stage = one K-tile of 128: both weight tiles (2 x 16 KB of shared
-// memory, 2 x 8 KB from HBM) and the unit's token rows of every term
-// (N x 128 bytes), all on one mbarrier; the MMA issuer runs 8 MMAs of K 32
-// and commits the stage back to the loader.  Scales travel in scale stages of
-// G K-tiles through tensor memory.
+// Pipeline stage = KPS (1 or 2) K-tiles of 128: per K-tile both weight tiles
+// (2 x 16 KB of shared memory, 2 x 8 KB from HBM) and the unit's token rows of
+// every term (N x 128 bytes), all on one mbarrier; the MMA issuer runs 8 MMAs
+// of K 32 per K-tile and commits the stage back to the loader.  Scales travel
+// in scale stages of G K-tiles through tensor memory.
 //
 // Roles (320 threads, one CTA per SM, persistent over units):
 //   warps 0-3  epilogue (TMEM lane quadrant = warp): tcgen05.ld of the two
@@ -201,29 +201,6 @@ __device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Copies issued from a warp that runs the loader loop as a whole: every lane
-// calls with the same operands and only the lane whose `leader` is nonzero
-// (chosen once with elect.sync) issues, which keeps the operands warp-uniform.
-__device__ __forceinline__ uint32_t elect_leader() {
-  uint32_t r;
-  asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx_if(uint32_t leader, uint64_t* bar, uint32_t bytes) {
-  asm volatile("{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n}\n" ::"r"(
-                   leader),
-               "r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void tma_load_3d_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y, int z,
-                                               uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
-      " @e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%1], [%2, "
-      "{%3, %4, %5}], [%6], %7;\n}\n" ::"r"(leader),
-      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_3d_nohint_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y,
                                                       int z, uint64_t* bar) {
   asm volatile(

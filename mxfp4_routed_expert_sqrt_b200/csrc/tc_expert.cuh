@@ -196,6 +196,39 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Copies issued from a warp that runs the loader loop as a whole: every lane
+// calls with the same operands and only the lane whose `leader` is nonzero
+// (chosen once with elect.sync) issues, which keeps the operands warp-uniform.
+__device__ __forceinline__ uint32_t elect_leader() {
+  uint32_t r;
+  asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_if(uint32_t leader, uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n}\n" ::"r"(
+                   leader),
+               "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y, int z,
+                                               uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%1], [%2, "
+      "{%3, %4, %5}], [%6], %7;\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_if(uint32_t leader, void* dst, const CUtensorMap* map, int x, int y,
+                                               uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n setp.ne.b32 e, %0, 0;\n"
+      " @e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%1], [%2, {%3, %4}], "
+      "[%5];\n}\n" ::"r"(leader),
+      "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // f16x2 with 2^k in both halves, k in [-24, 15] (subnormal f16 below -14).
 __device__ __forceinline__ uint32_t pow2_f16x2(int k) {
   const float f = __uint_as_float((uint32_t)(k + 127) << 23);
@@ -585,12 +618,16 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     }
   } else if (warp == 14) {
     // ------------------------------ weight loader ------------------------------
-    if (lane == 0) {
+    // The whole warp runs the loop (wait outcomes agreed with __all_sync); one
+    // elected lane issues every copy and barrier arrival.
+    {
+      const uint32_t leader = elect_leader();
+      auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
       TcRing rw(args.w_slots);
       const uint64_t pol = policy_evict_first();
       const int n_slots = nst / args.st_per_slot;
       int issued = 0;
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && !warp_aborted(); u += gridDim.x) {
         if (u + (int)gridDim.x >= n_units) griddep_launch();  // this CTA's last unit
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
@@ -598,22 +635,24 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
         const int y0 = MODE == 0 ? mt * 128 : mt * 256;
         const int y1 = MODE == 0 ? mt * 128 : mt * 256 + 128;
         for (int i = 0; i < n_slots; ++i) {
-          if (!mbar_wait(&w_empty[rw.s], rw.ph ^ 1)) {
-            give_up();
+          if (!warp_wait(&w_empty[rw.s], rw.ph ^ 1)) {
+            if (lane == 0) give_up();
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&w_full[rw.s], (uint32_t)args.w_slot_bytes);
+          mbar_arrive_expect_tx_if(leader, &w_full[rw.s], (uint32_t)args.w_slot_bytes);
           uint8_t* dst = s_w + rw.s * args.w_slot_bytes;
           if (AF == kAMxfp4) {  // code bytes [i * w_inner, +w_inner) of 128 rows, expert e
-            tma_load_3d(dst, &wmap0, i * args.w_inner, y0, e, &w_full[rw.s], pol);
-            tma_load_3d(dst + tile_bytes, MODE == 0 ? &wmap1 : &wmap0, i * args.w_inner, y1, e, &w_full[rw.s], pol);
+            tma_load_3d_if(leader, dst, &wmap0, i * args.w_inner, y0, e, &w_full[rw.s], pol);
+            tma_load_3d_if(leader, dst + tile_bytes, MODE == 0 ? &wmap1 : &wmap0, i * args.w_inner, y1, e,
+                           &w_full[rw.s], pol);
           } else {  // bf16 columns (k mod a_cols) of the stage's two k-blocks
 #pragma unroll
             for (int g = 0; g < kTcKG; ++g) {
               const int x = (i * kTcStageK + g * kTcKB) % args.a_cols;
-              tma_load_3d(dst + g * 16384, &wmap0, x, y0, 0, &w_full[rw.s], pol);
-              tma_load_3d(dst + tile_bytes + g * 16384, MODE == 0 ? &wmap1 : &wmap0, x, y1, 0, &w_full[rw.s], pol);
+              tma_load_3d_if(leader, dst + g * 16384, &wmap0, x, y0, 0, &w_full[rw.s], pol);
+              tma_load_3d_if(leader, dst + tile_bytes + g * 16384, MODE == 0 ? &wmap1 : &wmap0, x, y1, 0,
+                             &w_full[rw.s], pol);
             }
           }
           rw.next();
@@ -625,33 +664,36 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       // path the A producers have already waited for every one of them)
       for (int i = 0; i < min(issued, rw.n); ++i) {
         const int s = (rw.s - 1 - i + rw.n) % rw.n;
-        if (!mbar_wait(&w_full[s], s < rw.s ? rw.ph : rw.ph ^ 1)) set_error(kErrWaitTc);
+        if (!warp_wait(&w_full[s], s < rw.s ? rw.ph : rw.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
       }
     }
     __syncwarp();
   } else if (warp == 12) {
     // ------------------------------ token loader -------------------------------
-    if (lane == 0) {
+    // the whole warp runs the loop; one elected lane issues
+    {
+      const uint32_t leader = elect_leader();
+      auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
       TcRing rs(args.stages);
       int issued = 0;
-      for (int u = blockIdx.x; u < n_units && !aborted(); u += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && !warp_aborted(); u += gridDim.x) {
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         bool ok = true;
         for (int st = 0; st < nst; ++st) {
-          if (!mbar_wait(&empty[rs.s], rs.ph ^ 1)) {
-            give_up();
+          if (!warp_wait(&empty[rs.s], rs.ph ^ 1)) {
+            if (lane == 0) give_up();
             ok = false;
             break;
           }
           // one box of n_chunk token rows per k-block (rows past the unit's
           // tokens are loaded but never stored)
-          mbar_arrive_expect_tx(&b_full[rs.s], (uint32_t)(kTcKG * NC * 128));
+          mbar_arrive_expect_tx_if(leader, &b_full[rs.s], (uint32_t)(kTcKG * NC * 128));
           uint8_t* dst = s_b + rs.s * bst;
 #pragma unroll
           for (int g = 0; g < kTcKG; ++g) {
             const int col = (st * kTcStageK + g * kTcKB) % args.b_cols;
-            tma_load_2d(dst + g * atom, &bmap, col, pos0, &b_full[rs.s]);
+            tma_load_2d_if(leader, dst + g * atom, &bmap, col, pos0, &b_full[rs.s]);
           }
           rs.next();
           ++issued;
@@ -660,7 +702,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       }
       for (int i = 0; i < min(issued, rs.n); ++i) {
         const int s = (rs.s - 1 - i + rs.n) % rs.n;
-        if (!mbar_wait(&b_full[s], s < rs.s ? rs.ph : rs.ph ^ 1)) set_error(kErrWaitTc);
+        if (!warp_wait(&b_full[s], s < rs.s ? rs.ph : rs.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
       }
     }
     __syncwarp();

@@ -294,7 +294,7 @@ EXPERT_DTYPES = {
 
 def expert_path(dims, B):
     avg = -(-B * dims.top_k // dims.n_experts)
-    return "block_scaled" if avg <= 8 else "dequant"
+    return "block_scaled" if avg <= 24 else "dequant"
 
 
 def kernel_source_hash(path):

@@ -206,7 +206,7 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *           dequantising path uses a prefix, so the size grows with T and a
  *           workspace sized for some T serves every smaller T.
  * Two paths, chosen from T alone (mean pairs per expert, ceil(T*top_k / E)):
- *  - at most 8 (decode): block-scaled tensor-core MMAs
+ *  - at most 24 (decode, small batches): block-scaled tensor-core MMAs
  *    (tcgen05 kind::mxf8f6f4): the E2M1 codes and E8M0 scales go to the
  *    tensor core as stored and are applied there.  Each activation enters as
  *    two E4M3 terms with E8M0 group-32 scales (a bf16 x is carried exactly
@@ -215,7 +215,7 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
  *    Workspace: E4M3 terms and E8M0 scales of x in expert order
  *    [2][T*top_k][hidden] and [2][T*top_k][hidden/32], then of h
  *    [3][T*top_k][inter] and [3][T*top_k][inter/32] bytes.
- *  - above 8 (prefill): each weight is dequantised to f16 times a power of
+ *  - above 24 (prefill): each weight is dequantised to f16 times a power of
  *    two per weight row (undone in fp32): exactly for every E8M0 group within
  *    36 octaves of the largest group of its row, whatever the bytes; groups
  *    further below are flushed to zero (their products lie below 2^-36 of

@@ -23,13 +23,19 @@ inline int expert_chunk(int T, int K, int E) {
 }
 
 // Mean pairs per expert up to which moe_expert_gemm takes the block-scaled
-// kernel; above it, the kernel that dequantises to f16.
-constexpr int kBlockScaledMaxAvg = 8;
+// kernel; above it, the kernel that dequantises to f16.  Measured on one B200
+// (expert call, same box): at 8, 12, 16, 20 and 24 pairs per expert the
+// block-scaled kernel in 32-pair chunks takes 762 / 777 / 808 / 842 / 890 us
+// against 1319 / 1323 / 1329 / 1334 / 1341 us dequantising; at 32, 48, 64 and
+// 96 the dequantising kernel wins (1393 / 1422 / 1469 / 1605 us against 1788 /
+// 1987 / 2161 / 2544 us for the block-scaled kernel's summed layout).
+constexpr int kBlockScaledMaxAvg = 24;
 
 // Path choice from the host-known T: with few pairs per expert (32-pair
-// chunks, decode) the weights stream through the block-scaled kernel; with
-// many, the kernel that dequantises to f16 keeps 128-token units, double the
-// epilogue warps and one read of each expert's weights.
+// chunks: decode and small batches) the weights stream through the
+// block-scaled kernel; with many, the kernel that dequantises to f16 keeps
+// 128-token units, double the epilogue warps and one read of each expert's
+// weights.
 inline bool use_block_scaled(int T, int K, int E) {
   return ((int64_t)T * K + E - 1) / E <= kBlockScaledMaxAvg;
 }
@@ -39,13 +45,13 @@ inline bool use_block_scaled(int T, int K, int E) {
 constexpr int kXTerms = 2;
 constexpr int kHTerms = 3;
 
-// Token layout of the block-scaled kernel by mean pairs per expert: up to 8,
-// the terms stacked along N in 32-pair chunks (N 64 and 96 cost what N 16
-// does) with one accumulator set; up to 24, the terms summed into one
-// accumulator in 64-pair chunks with two accumulator sets (a unit's epilogue
-// overlaps the next unit's MMAs); above, 128-pair chunks (N 128, the MMA's
-// efficient width; one set fits), so an expert's weights are read once per
-// 128 of its pairs.
+// Token layout of the block-scaled kernel by mean pairs per expert: on its
+// path (up to kBlockScaledMaxAvg), the terms stacked along N in 32-pair chunks
+// (N 64 and 96 cost about what N 16 does) with two accumulator sets; an
+// expert with more than 32 pairs takes more chunks.  Above, the layout the
+// kernel was measured in against the dequantising one at prefill (not on any
+// path): the terms summed into one accumulator in 128-pair chunks (N 128;
+// one set fits), so an expert's weights are read once per 128 of its pairs.
 struct MxLayout {
   int chunk, term_acc, max_bufs;
 };
@@ -55,8 +61,7 @@ struct MxLayout {
 constexpr int kMxDecodeBufs = 2;  // accumulator sets of the stacked (decode) layout
 inline MxLayout mx_layout(int T, int K, int E) {
   const int64_t avg = ((int64_t)T * K + E - 1) / E;
-  if (avg <= 8) return {32, 0, kMxDecodeBufs};
-  if (avg <= 24) return {64, 1, 2};
+  if (avg <= kBlockScaledMaxAvg) return {32, 0, kMxDecodeBufs};
   return {128, 1, 2};
 }
 

@@ -1,6 +1,7 @@
 // Grouped MXFP4 expert GEMM on the block-scaled tensor cores
 // (tcgen05.mma.kind::mxf8f6f4.block_scale): the path of moe_expert_gemm for
-// calls with at most 8 pairs per expert on average (decode).
+// calls with at most 24 pairs per expert on average (decode and small
+// batches).
 //
 // The weights reach the MMA exactly as stored: E2M1 codes straight from HBM by
 // TMA (CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, which widens every 8 bytes of

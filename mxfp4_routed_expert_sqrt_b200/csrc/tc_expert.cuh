@@ -1,6 +1,6 @@
 // Grouped expert GEMM on the 5th-generation tensor cores (tcgen05) with the
 // weights dequantised in software: moe_expert_gemm's path for calls with more
-// than 8 pairs per expert on average (prefill), and the bf16 GEMMs of the
+// than 24 pairs per expert on average (prefill), and the bf16 GEMMs of the
 // router and the shared expert above 64 tokens.
 //
 // Per unit = (expert e, token chunk of <= n_chunk grouped pairs, row tile):

@@ -61,7 +61,7 @@ def expert_call(T, bad_perm=False, bad_offsets=False):
     torch.cuda.synchronize()
     return m.moe_device_error()
 
-for T, path in ((8, "block_scaled"), (100, "dequant")):
+for T, path in ((8, "block_scaled"), (200, "dequant")):  # 1 and 25 pairs per expert
     res[f"{path}_valid"] = expert_call(T)
     res[f"{path}_bad_perm"] = expert_call(T, bad_perm=True)
     res[f"{path}_bad_offsets"] = expert_call(T, bad_offsets=True)

@@ -183,20 +183,23 @@ def _expert_gemm(dc, T):
 
 
 # The call picks its path and token chunk from the mean pairs per expert: at
-# most 8 runs the block-scaled kernel in 32-pair chunks (every case here up to
-# v4_T300 and the tiny T8/T37 ones), more runs the dequantising kernel in 64-
-# or 128-pair chunks (tiny T100/T1000).  The zipf case piles most pairs onto a
-# few experts, so their groups span many 32-pair chunks, and it samples both
-# sides of every chunk boundary of the most loaded expert.
+# most 24 runs the block-scaled kernel in 32-pair chunks (every case here up
+# to v4_T1024 and the tiny T8/T37/T100 ones), more runs the dequantising
+# kernel in 128-pair chunks (tiny T200/T1000, v4_T1025, the prefill size).
+# The zipf case piles most pairs onto a few experts, so their groups span many
+# 32-pair chunks, and it samples both sides of every chunk boundary of the
+# most loaded expert.
 EXPERT_CASES = [("tiny_T8", gen.TINY, 8, 64, None), ("tiny_T37", gen.TINY, 37, 74, None),
                 ("v4_T1", gen.V4, 1, 6, None), ("v4_T8", gen.V4, 8, 48, None), ("v4_T37", gen.V4, 37, 24, None),
-                ("v4_T64", gen.V4, 64, 24, None), ("tiny_T100_tc", gen.TINY, 100, 200, None),
-                ("tiny_T1000_tc", gen.TINY, 1000, 120, None), ("v4_T96_tc", gen.V4, 96, 24, None),
-                ("v4_T300_tc", gen.V4, 300, 24, None), ("v4_zipf_T256_chunks", gen.V4, 256, 16, "zipf"),
-                # the two sides of the path switch: 8 pairs per expert on average
-                # (the largest block-scaled call), then 9 (the smallest dequantising one)
-                ("v4_T341_block_scaled_max", gen.V4, 341, 24, None),
-                ("v4_T342_dequant_min", gen.V4, 342, 24, None),
+                ("v4_T64", gen.V4, 64, 24, None), ("tiny_T100", gen.TINY, 100, 200, None),
+                ("tiny_T200_tc", gen.TINY, 200, 200, None), ("tiny_T1000_tc", gen.TINY, 1000, 120, None),
+                ("v4_T96", gen.V4, 96, 24, None), ("v4_T300", gen.V4, 300, 24, None),
+                ("v4_zipf_T256_chunks", gen.V4, 256, 16, "zipf"),
+                # the two sides of the path switch: 24 pairs per expert on average
+                # (the largest block-scaled call, many experts past one 32-pair
+                # chunk), then 25 (the smallest dequantising one)
+                ("v4_T1024_block_scaled_max", gen.V4, 1024, 32, None),
+                ("v4_T1025_dequant_min", gen.V4, 1025, 24, None),
                 # the prefill size: 256 pairs spread over the call plus every pair of
                 # the four most loaded experts (each of their chunk positions)
                 ("v4_T4096_prefill", gen.V4, 4096, 256, "chunks")]

@@ -284,7 +284,8 @@ struct TcArgs {
   float limit;
   // pipeline shape, filled in by tc_plan()
   int acc_cols;      // TMEM columns per accumulator (>= n_chunk)
-  int stages;        // pipeline stages (TMEM A + token tiles of 2 k-blocks)
+  int stages;        // pipeline stages (TMEM A of 2 k-blocks)
+  int b_stages;      // token-tile ring (shared memory, 2 k-blocks each): may run ahead of the TMEM stages
   int w_slots;       // weight slots
   int w_inner;       // bytes of one weight row in one TMA box
   int w_slot_bytes;  // bytes of one weight slot (both tiles)
@@ -326,11 +327,36 @@ inline bool tc_plan(TcArgs& a, int af) {
   const int groups = a.offsets != nullptr ? a.E : 1;
   const int pre = (2 * (groups + 1) * 4 + 127) / 128 * 128;  // unit prefix + group offsets
   const int budget = kTcSmemMax - 1024;  // 1024: alignment slack of the dynamic base
-  const int w = (budget - a.stages * bst - sc - pre) / a.w_slot_bytes;
+  auto weight_slots = [&](int b_stages) { return (budget - b_stages * bst - sc - pre) / a.w_slot_bytes; };
+  // Token tiles one stage deeper than the TMEM stages, so a tile's copy is in
+  // flight while the two TMEM stages turn over (its latency otherwise stalls
+  // every stage): MXFP4 weights then come in 64-byte boxes (one stage per
+  // slot) if 128-byte ones leave no room for it.  At least three weight stages
+  // stay in flight.
+  a.b_stages = a.stages;
+  if (af == kAMxfp4 && a.stages + 1 <= kTcMaxStages) {
+    const int b3 = a.stages + 1;
+    if (weight_slots(b3) * a.st_per_slot >= 3 && weight_slots(b3) >= 2) {
+      a.b_stages = b3;
+    } else if (a.w_inner == 128 && (a.a_cols / 2) % 64 == 0) {
+      const int keep_inner = a.w_inner, keep_sps = a.st_per_slot, keep_wsb = a.w_slot_bytes;
+      a.w_inner = 64;
+      a.st_per_slot = 1;
+      a.w_slot_bytes = 2 * 128 * 64;
+      if (weight_slots(b3) >= 3) {
+        a.b_stages = b3;
+      } else {
+        a.w_inner = keep_inner;
+        a.st_per_slot = keep_sps;
+        a.w_slot_bytes = keep_wsb;
+      }
+    }
+  }
+  const int w = weight_slots(a.b_stages);
   a.w_slots = w < 6 ? w : 6;
   if (a.w_slots < 2) return false;
   a.off_b = a.w_slots * a.w_slot_bytes;
-  a.off_sc = a.off_b + a.stages * bst;
+  a.off_sc = a.off_b + a.b_stages * bst;
   a.off_prefix = a.off_sc + sc;
   a.smem_bytes = a.off_prefix + pre + 1024;
   return a.smem_bytes <= kTcSmemMax;
@@ -341,7 +367,8 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     tc_expert_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap0,
                      const __grid_constant__ CUtensorMap wmap1, const TcArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages], b_full[kTcMaxStages];
+  __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages];
+  __shared__ __align__(8) uint64_t b_full[kTcMaxStages], b_empty[kTcMaxStages];
   __shared__ __align__(8) uint64_t w_full[kTcMaxStages], w_empty[kTcMaxStages];
   __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
   __shared__ uint32_t s_taddr;
@@ -350,7 +377,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_w = smem;                  // weight ring
-  uint8_t* s_b = smem + args.off_b;     // token tiles, one per stage
+  uint8_t* s_b = smem + args.off_b;     // token tiles, ring of b_stages
   uint8_t* s_sc = smem + args.off_sc;   // E8M0 rows, two unit buffers, thread-major
   int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + args.off_prefix);  // [E + 1] units before group e
   int32_t* s_off = s_prefix + (args.offsets != nullptr ? args.E : 1) + 1;  // [E + 1] copy of offsets
@@ -405,9 +432,10 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
   }
   if (tid == 0) {
     for (int s = 0; s < kTcMaxStages; ++s) {
-      mbar_init(&full[s], 8);  // one arrival per A-producer warp (one of them also waits for the tokens)
+      mbar_init(&full[s], 8);  // one arrival per A-producer warp
       mbar_init(&empty[s], 1);
       mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
       mbar_init(&w_full[s], 1);
       mbar_init(&w_empty[s], 8);
     }
@@ -464,14 +492,11 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     const uint32_t mask = (uint32_t)args.w_inner / 16 - 1;
     TcRing rs(args.stages), rw(args.w_slots);
     int js = 0;  // stage within the current weight slot
-    // publish stage rs.s (both k-blocks stored): the tokens of the stage must
-    // have landed too (warp 4 checks), then one arrival per warp
-    auto publish = [&]() -> bool {
+    // publish stage rs.s (both k-blocks stored): one arrival per warp
+    auto publish = [&]() {
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      bool ok = true;
-      if (warp == 4 && lane == 0) ok = mbar_wait(&b_full[rs.s], rs.ph);
       if (lane == 0) mbar_arrive(&full[rs.s]);
       rs.next();
       if (++js == args.st_per_slot) {  // slot fully read: hand it back to the loader
@@ -479,7 +504,6 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
         if (lane == 0) mbar_arrive(&w_empty[rw.s]);
         rw.next();
       }
-      return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
     auto wait_stage = [&]() -> bool {  // TMEM stage free (its MMAs done)
       if (!warp_wait(&empty[rs.s], rs.ph ^ 1)) return false;
@@ -562,16 +586,18 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
             break;
           }
           const uint32_t sw = sc_word(st);  // E8M0 of this stage's two k-blocks
+          // both k-blocks converted while the stage is still in use: once it
+          // frees, only the stores stand between it and the MMAs
           uint32_t v0[32], v1[32];
           convert(0, sw, v0);
+          convert(1, sw, v1);
           if (!wait_stage()) {
             ok = false;
             break;
           }
           tmem_st32(tl + rs.s * kTcStageCols, v0);
-          convert(1, sw, v1);
           tmem_st32(tl + rs.s * kTcStageCols + 64, v1);
-          ok = publish();
+          publish();
         }
         if (!ok) {
           give_up();
@@ -601,14 +627,14 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
           }
           uint32_t v0[32], v1[32];
           copy(0, v0);
+          copy(1, v1);
           if (!wait_stage()) {
             ok = false;
             break;
           }
           tmem_st32(tl + rs.s * kTcStageCols, v0);
-          copy(1, v1);
           tmem_st32(tl + rs.s * kTcStageCols + 64, v1);
-          ok = publish();
+          publish();
         }
         if (!ok) {
           give_up();
@@ -674,35 +700,35 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     {
       const uint32_t leader = elect_leader();
       auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
-      TcRing rs(args.stages);
+      TcRing rb(args.b_stages);  // token tiles, released by the MMAs that read them
       int issued = 0;
       for (int u = blockIdx.x; u < n_units && !warp_aborted(); u += gridDim.x) {
         int e, mt, pos0, n;
         decode_unit(u, e, mt, pos0, n);
         bool ok = true;
         for (int st = 0; st < nst; ++st) {
-          if (!warp_wait(&empty[rs.s], rs.ph ^ 1)) {
+          if (!warp_wait(&b_empty[rb.s], rb.ph ^ 1)) {
             if (lane == 0) give_up();
             ok = false;
             break;
           }
           // one box of n_chunk token rows per k-block (rows past the unit's
           // tokens are loaded but never stored)
-          mbar_arrive_expect_tx_if(leader, &b_full[rs.s], (uint32_t)(kTcKG * NC * 128));
-          uint8_t* dst = s_b + rs.s * bst;
+          mbar_arrive_expect_tx_if(leader, &b_full[rb.s], (uint32_t)(kTcKG * NC * 128));
+          uint8_t* dst = s_b + rb.s * bst;
 #pragma unroll
           for (int g = 0; g < kTcKG; ++g) {
             const int col = (st * kTcStageK + g * kTcKB) % args.b_cols;
-            tma_load_2d_if(leader, dst + g * atom, &bmap, col, pos0, &b_full[rs.s]);
+            tma_load_2d_if(leader, dst + g * atom, &bmap, col, pos0, &b_full[rb.s]);
           }
-          rs.next();
+          rb.next();
           ++issued;
         }
         if (!ok) break;
       }
-      for (int i = 0; i < min(issued, rs.n); ++i) {
-        const int s = (rs.s - 1 - i + rs.n) % rs.n;
-        if (!warp_wait(&b_full[s], s < rs.s ? rs.ph : rs.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
+      for (int i = 0; i < min(issued, rb.n); ++i) {
+        const int s = (rb.s - 1 - i + rb.n) % rb.n;
+        if (!warp_wait(&b_full[s], s < rb.s ? rb.ph : rb.ph ^ 1) && lane == 0) set_error(kErrWaitTc);
       }
     }
     __syncwarp();
@@ -712,7 +738,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
     // it stays converged); an elected lane issues each MMA and commit.
     // Descriptors are built once and advanced by byte offset / 16 (operands
     // lie below 256 KB: the 14-bit address field never carries).
-    TcRing rs(args.stages);
+    TcRing rs(args.stages), rb(args.b_stages);
     uint32_t un = 0;
     const uint64_t d_b = sdesc_sw128(smem_u32(s_b));
     auto warp_aborted = [&]() { return __shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0) != 0; };
@@ -729,12 +755,12 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
       }
       tc_fence_after();
       for (int st = 0; st < nst; ++st) {
-        if (!warp_wait(&full[rs.s], rs.ph)) {
+        if (!warp_wait(&full[rs.s], rs.ph) || !warp_wait(&b_full[rb.s], rb.ph)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t bd0 = d_b + (uint64_t)((rs.s * bst) >> 4);
+        const uint64_t bd0 = d_b + (uint64_t)((rb.s * bst) >> 4);
         const uint32_t a0 = tbase + a_base + rs.s * kTcStageCols;
         const uint32_t acc1 = tbase + args.acc_cols;
         const uint32_t first = st > 0 ? 1u : 0u;
@@ -750,8 +776,10 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
           }
         }
         umma_commit_warp(&empty[rs.s]);
+        umma_commit_warp(&b_empty[rb.s]);
         if (st == nst - 1) umma_commit_warp(&acc_full);
         rs.next();
+        rb.next();
       }
       if (!ok) break;
     }

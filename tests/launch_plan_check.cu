@@ -77,6 +77,14 @@ static void check_tc_plan(TcArgs a, const char* name, int T) {
   CHECK(a.acc_cols >= a.n_chunk, "%s T=%d", name, T);
   CHECK(2 * a.acc_cols + a.stages * kTcStageCols <= kTcTmemCols, "%s T=%d TMEM", name, T);
   CHECK(a.stages >= 2 && a.w_slots >= 2, "%s T=%d rings", name, T);
+  // the token ring runs at least as deep as the TMEM stages, and one deeper
+  // with at least three weight stages in flight where the shared memory allows
+  CHECK(a.b_stages >= a.stages && a.b_stages <= kTcMaxStages, "%s T=%d token ring", name, T);
+  CHECK(a.b_stages == a.stages || a.w_slots * a.st_per_slot >= 3, "%s T=%d weight stages", name, T);
+  CHECK(a.st_per_slot * 64 == a.w_inner && (a.a_cols / 2) % a.w_inner == 0, "%s T=%d weight box", name, T);
+  // shared memory: weight slots, then the token ring, the E8M0 rows, the prefix
+  CHECK(a.off_b == a.w_slots * a.w_slot_bytes && a.off_sc == a.off_b + a.b_stages * kTcKG * a.n_chunk * 128,
+        "%s T=%d offsets", name, T);
   CHECK(a.smem_bytes <= kTcSmemMax && 2 * a.smem_bytes > kTcSmemMax, "%s T=%d smem %d", name, T, a.smem_bytes);
 }
 

@@ -147,8 +147,13 @@ bool make_weight_map(CUtensorMap* map, const uint8_t* base, int af, const TcArgs
   }
   box[1] = 128;
   box[2] = 1;
+  // a 64-byte box reads half of a row's 128-byte line; the next stage's box
+  // reads the other half, so L2 fills go by 128 bytes, not 256
+  const CUtensorMapL2promotion promo =
+      box[0] * (type == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 ? 2 : 1) >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                                                         : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
   return fn(map, type, 3, const_cast<uint8_t*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Plans the pipeline of one tensor-core expert launch, builds its weight

@@ -810,11 +810,22 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
         s1 = pow2_f32(s_crow[un % kCrowRing][1][r]);
       }
       float hmax = 0.f;  // MXFP4 gate/up: the largest |h| of this warp's rows in the unit
+      // the accumulator is handed back to the MMA warp as soon as this warp's
+      // last columns are in registers (before their SwiGLU and stores): the
+      // next unit's MMAs overwrite it
+      bool released = false;
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty);
+        released = true;
+      };
       for (int c0 = 16 * half; c0 < n; c0 += 16 * (EPI / 4)) {
         uint32_t g[16], h[16];
         tmem_ld16(tbase + lrow + c0, g);
         tmem_ld16(tbase + lrow + args.acc_cols + c0, h);
         tmem_ld_wait();
+        if (c0 + 16 * (EPI / 4) >= n) release();
         if (MODE == 0) {
           const int col = mt * 128 + r;
 #pragma unroll
@@ -850,9 +861,7 @@ __global__ void __launch_bounds__(tc_threads(EPI), 1)
         const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(hmax)));
         if (lane == 0 && m > 0.f && m < 6.103515625e-05f) set_error(kErrF16Small);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty);
+      if (!released) release();  // a warp with no columns in this unit
     }
   }
 

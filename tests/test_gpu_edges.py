@@ -191,3 +191,20 @@ def test_layer_with_every_activation_edge():
     want, _, _ = oracle.moe_layer(V4, c.x, sel, c.router, None, gb, ub, db, shared=c.shared)
     mx, mean = rel_errors(got[sel], want)
     assert mx <= MAX_TOL and mean <= MEAN_TOL, f"max {mx:.2e} mean {mean:.2e}"
+
+
+def test_dequant_path_flags_a_row_span_beyond_f16():
+    """Groups 44 octaves apart inside a weight row (E8M0 bytes drawn per group
+    from [96, 140]) cannot all be exact in f16 on the dequantising path: the
+    groups more than 36 octaves below their row's largest are flushed and the
+    call records 0x302 (include/moe.h).  The block-scaled path applies the
+    scales in the MMA and records nothing.  (Such rows are ill-conditioned for
+    any fp32 accumulator near the SwiGLU kink, so only the status is checked.)"""
+    for T, want in ((1100, m.DEVICE_ERR_SPAN_FLUSH), (8, 0)):
+        assert _dequant_path(T) == (want != 0)
+        c = make_case(V4, T, seed=11, with_shared=False, e_range=(96, 140))
+        dc = DeviceCase(c, DEV)
+        _, _, y = _expert_gemm(dc, T)
+        assert m.moe_device_error() == want, f"T={T}"
+        if want == 0:
+            assert np.isfinite(y).all()

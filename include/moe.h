@@ -193,6 +193,13 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t K, int32_t E,
 size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T);
 
 /*
+ * The path moe_expert_gemm takes for T tokens (host only, no GPU work):
+ * 1 = block-scaled tensor-core MMAs, 0 = dequantising to f16 (see below);
+ * -MOE_ERR_INVALID_ARG for a null dims, invalid dims or T < 0.
+ */
+int32_t moe_expert_gemm_path(const moe_dims* dims, int32_t T);
+
+/*
  * All routed experts for the grouped pairs:
  *   y_perm[pos] = Wd_e (silu(min(Wg_e x_t, L)) * clamp(Wu_e x_t, -L, L))
  * for pos in [offsets[e], offsets[e+1]), p = perm[pos], t = p / top_k.

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3
 EXPORTS = ("moe_abi_version", "moe_status_string", "moe_device_error", "moe_selftest_wait",
            "moe_route_workspace_size",
            "moe_route", "moe_route_noalloc", "moe_permute_workspace_size", "moe_permute",
-           "moe_expert_gemm_workspace_size", "moe_expert_gemm", "shared_expert_workspace_size",
+           "moe_expert_gemm_workspace_size", "moe_expert_gemm_path", "moe_expert_gemm", "shared_expert_workspace_size",
            "shared_expert", "moe_combine")
 
 
@@ -79,6 +79,8 @@ def lib():
         L.moe_permute.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_expert_gemm_workspace_size.restype = _sz
         L.moe_expert_gemm_workspace_size.argtypes = [dp, _i32]
+        L.moe_expert_gemm_path.restype = _i32
+        L.moe_expert_gemm_path.argtypes = [dp, _i32]
         L.moe_expert_gemm.restype = ctypes.c_int
         L.moe_expert_gemm.argtypes = [dp, _vp, _i32, moe_mxfp4_proj, moe_mxfp4_proj, moe_mxfp4_proj,
                                       _vp, _vp, _vp, _vp, _sz, _vp]
@@ -193,6 +195,14 @@ def moe_permute(topk_idx, T, K, E, offsets, perm, inv, ws=None, ws_bytes=0, stre
 
 def moe_expert_gemm_workspace_size(dims, T) -> int:
     return lib().moe_expert_gemm_workspace_size(ctypes.byref(dims_of(dims)), T)
+
+
+def moe_expert_gemm_path(dims, T) -> str:
+    """'block_scaled' or 'dequant': the path moe_expert_gemm takes for T tokens."""
+    r = lib().moe_expert_gemm_path(ctypes.byref(dims_of(dims)), T)
+    if r < 0:
+        raise MoeError("moe_expert_gemm_path", -r)
+    return "block_scaled" if r == 1 else "dequant"
 
 
 def moe_expert_gemm(dims, x, T, gate, up, down, offsets, perm, y_perm, ws, ws_bytes, stream=None):

@@ -512,6 +512,11 @@ size_t moe_expert_gemm_workspace_size(const moe_dims* dims, int32_t T) {
   return expert_gemm_ws_bytes(*dims, T);
 }
 
+int32_t moe_expert_gemm_path(const moe_dims* dims, int32_t T) {
+  if (check_dims(dims) != MOE_OK || T < 0) return -(int32_t)MOE_ERR_INVALID_ARG;
+  return use_block_scaled(T, dims->top_k, dims->n_experts) ? 1 : 0;
+}
+
 namespace {
 
 moe_status expert_gemm_block_scaled(const moe_dims* dims, const void* x, int32_t T, const moe_mxfp4_proj& gate,

@@ -149,3 +149,19 @@ def test_permute_argument_errors(m):
     with pytest.raises(m.MoeError) as e:
         m.moe_permute(1 << 40, 1 << 21, 6, 256, 1 << 40, 1 << 40, 1 << 40)
     assert e.value.status == 3
+
+
+def test_expert_path_choice(m):
+    """moe_expert_gemm's path for T (host only): block-scaled up to 24 pairs
+    per expert on average, dequantising above; bench.py's mirror of the switch
+    (which labels its roofline line) agrees for every T."""
+    import bench
+    assert m.moe_expert_gemm_path(gen.V4, 1024) == "block_scaled"
+    assert m.moe_expert_gemm_path(gen.V4, 1025) == "dequant"
+    assert m.moe_expert_gemm_path(gen.TINY, 192) == "block_scaled"
+    assert m.moe_expert_gemm_path(gen.TINY, 193) == "dequant"
+    for dims in (gen.V4, gen.TINY):
+        for T in list(range(0, 1300)) + [2048, 4096, 65536]:
+            assert m.moe_expert_gemm_path(dims, T) == bench.expert_path(dims, T), (dims, T)
+    with pytest.raises(m.MoeError):
+        m.moe_expert_gemm_path(gen.V4, -1)

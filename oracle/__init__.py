@@ -49,6 +49,14 @@ def lib():
         L.oracle_swiglu.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_double]
         L.oracle_dequant.restype = None
         L.oracle_dequant.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, _dp]
+        L.oracle_affine_expert_bytes.restype = ctypes.c_int64
+        L.oracle_affine_expert_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+        L.oracle_affine_dequant.restype = ctypes.c_int
+        L.oracle_affine_dequant.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp]
+        L.oracle_affine_expert_ffn.restype = ctypes.c_int
+        L.oracle_affine_expert_ffn.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int,
+                                               _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_double, _dp, ctypes.c_int, _dp]
         L.oracle_route.restype = None
         L.oracle_route.argtypes = [_u16p, ctypes.c_int, ctypes.c_int, _fp, _fp, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_double, _ip, _dp, _dp, _dp]
@@ -111,6 +119,32 @@ def dequant(blob: np.ndarray, rows: int, cols: int) -> np.ndarray:
     out = np.empty((rows, cols), dtype=np.float64)
     lib().oracle_dequant(_p(blob, _u8p), rows, cols, _p(out, _dp))
     return out
+
+
+def affine_expert_bytes(rows: int, cols: int, bits: int, group: int) -> int:
+    """Bytes of one affine-format expert blob (-1: a shape the format cannot hold)."""
+    return lib().oracle_affine_expert_bytes(rows, cols, bits, group)
+
+
+def affine_dequant(blob: np.ndarray, rows: int, cols: int, bits: int, group: int) -> np.ndarray:
+    """W = scale * q + bias of an affine blob, fp64 [rows][cols]."""
+    blob = _c(blob, np.uint8)
+    out = np.empty((rows, cols), dtype=np.float64)
+    if lib().oracle_affine_dequant(_p(blob, _u8p), rows, cols, bits, group, _p(out, _dp)) != 0:
+        raise ValueError("affine_dequant: bad shape")
+    return out
+
+
+def affine_expert_ffn(g, u, d, H, I, limit, xs):
+    """One affine expert on xs[n][H]; g, u, d = (blob, bits, group)."""
+    xs = _c(xs, np.float64)
+    n = xs.shape[0]
+    ys = np.empty((n, H), np.float64)
+    (gb, gbits, ggr), (ub, ubits, ugr), (db, dbits, dgr) = ((_c(b, np.uint8), bi, gr) for b, bi, gr in (g, u, d))
+    if lib().oracle_affine_expert_ffn(_p(gb, _u8p), gbits, ggr, _p(ub, _u8p), ubits, ugr, _p(db, _u8p), dbits, dgr,
+                                      H, I, limit, _p(xs, _dp), n, _p(ys, _dp)) != 0:
+        raise ValueError("affine_expert_ffn: bad shape")
+    return ys
 
 
 def route(x_bits, router_w, bias, K, alpha):

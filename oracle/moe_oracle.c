@@ -28,7 +28,9 @@
  *            base + xid * expert_bytes; E2M1 nibble plane plus E8M0 group-32
  *            scale plane.
  *  [JANG]    "DeepSeek-V4-Flash-0731-JANG", Dynamic affine recipe table: the
- *            router is kept in f32 (its weight is an fp32 input here).
+ *            router is kept in f32 (its weight is an fp32 input here); the
+ *            affine low-bit expert format (oracle_affine_*: the oracle step
+ *            of a variant whose CUDA path is not built).
  *
  * Readings where the pages are silent (each one a choice of this oracle):
  *  - nibble order: the low nibble of a byte is the even column;
@@ -87,6 +89,60 @@ static double bf16_to_double(uint16_t b) {
   float f;
   memcpy(&f, &u, 4);
   return (double)f;
+}
+
+/* ------------------------------------------------------------------ */
+/* Affine low-bit experts [JANG Dynamic affine recipe]: b-bit codes q in */
+/* [0, 2^b - 1] with one scale and one bias per group of G consecutive   */
+/* input columns of a row, w = scale * q + bias (2-bit G32 down, 2-bit   */
+/* G64 gate/up, 3-bit G64 gate in the lifted layers, 8-bit G64 shared).  */
+/* Readings (the page gives bits and group sizes per tensor role only):  */
+/*  - the codes of a row are one little-endian bit stream: column c      */
+/*    holds bits [c*b, c*b + b) of the row's cols*b/8 bytes, the lowest  */
+/*    bit first;                                                         */
+/*  - scales and biases are bf16;                                        */
+/*  - blob: codes [rows][cols*b/8], then scales [rows][cols/G], then     */
+/*    biases [rows][cols/G], experts back to back as for MXFP4.          */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of one affine expert blob; -1 for a shape the format cannot hold. */
+int64_t oracle_affine_expert_bytes(int64_t rows, int64_t cols, int bits, int group) {
+  if (rows <= 0 || bits < 1 || bits > 8 || group <= 0 || cols <= 0 || cols % group || (cols * bits) % 8 ||
+      (rows * cols * bits / 8) % 2)
+    return -1;
+  return rows * cols * bits / 8 + 2 * 2 * rows * (cols / group);
+}
+
+/* Code of column c from a row's bit stream, one bit at a time. */
+static int affine_code(const uint8_t* row_codes, int c, int bits) {
+  int q = 0;
+  for (int i = 0; i < bits; ++i) {
+    const int64_t bit = (int64_t)c * bits + i;
+    q |= ((row_codes[bit / 8] >> (bit % 8)) & 1) << i;
+  }
+  return q;
+}
+
+static void affine_dequant_row(const uint8_t* blob, int rows, int cols, int bits, int group, int r,
+                               double* out) {
+  const int64_t row_bytes = (int64_t)cols * bits / 8;
+  const uint8_t* codes = blob + (int64_t)r * row_bytes;
+  const uint8_t* scales = blob + (int64_t)rows * row_bytes;
+  const uint8_t* biases = scales + 2 * (int64_t)rows * (cols / group);
+  for (int c = 0; c < cols; ++c) {
+    const int64_t gi = (int64_t)r * (cols / group) + c / group;
+    uint16_t sb, bb;
+    memcpy(&sb, scales + 2 * gi, 2);
+    memcpy(&bb, biases + 2 * gi, 2);
+    out[c] = bf16_to_double(sb) * (double)affine_code(codes, c, bits) + bf16_to_double(bb);
+  }
+}
+
+/* W[r][c] of an affine blob into out[rows*cols]; -1 for a bad shape. */
+int oracle_affine_dequant(const uint8_t* blob, int rows, int cols, int bits, int group, double* out) {
+  if (oracle_affine_expert_bytes(rows, cols, bits, group) < 0) return -1;
+  for (int r = 0; r < rows; ++r) affine_dequant_row(blob, rows, cols, bits, group, r, out + (int64_t)r * cols);
+  return 0;
 }
 
 /* ------------------------------------------------------------------ */
@@ -247,6 +303,49 @@ void oracle_expert_ffn(const uint8_t* g_blob, const uint8_t* u_blob, const uint8
   free(wrow);
   free(g);
   free(u);
+}
+
+/*
+ * One affine expert on n activation rows xs[n][H] (fp64), ys[n][H] out: the
+ * same clamped SwiGLU FFN as oracle_expert_ffn with each projection in the
+ * affine format of its own bits and group size.  -1 for a bad shape.
+ */
+int oracle_affine_expert_ffn(const uint8_t* g_blob, int g_bits, int g_group, const uint8_t* u_blob, int u_bits,
+                             int u_group, const uint8_t* d_blob, int d_bits, int d_group, int H, int I,
+                             double limit, const double* xs, int n, double* ys) {
+  if (oracle_affine_expert_bytes(I, H, g_bits, g_group) < 0 || oracle_affine_expert_bytes(I, H, u_bits, u_group) < 0 ||
+      oracle_affine_expert_bytes(H, I, d_bits, d_group) < 0)
+    return -1;
+  double* wrow = (double*)malloc(sizeof(double) * (H > I ? H : I));
+  double* g = (double*)malloc(sizeof(double) * (int64_t)n * I);
+  double* u = (double*)malloc(sizeof(double) * (int64_t)n * I);
+  for (int r = 0; r < I; ++r) {
+    affine_dequant_row(g_blob, I, H, g_bits, g_group, r, wrow);
+    for (int j = 0; j < n; ++j) {
+      double acc = 0.0;
+      for (int c = 0; c < H; ++c) acc += wrow[c] * xs[(int64_t)j * H + c];
+      g[(int64_t)j * I + r] = acc;
+    }
+    affine_dequant_row(u_blob, I, H, u_bits, u_group, r, wrow);
+    for (int j = 0; j < n; ++j) {
+      double acc = 0.0;
+      for (int c = 0; c < H; ++c) acc += wrow[c] * xs[(int64_t)j * H + c];
+      u[(int64_t)j * I + r] = acc;
+    }
+  }
+  for (int64_t i = 0; i < (int64_t)n * I; ++i) g[i] = oracle_swiglu(g[i], u[i], limit);
+  for (int r = 0; r < H; ++r) {
+    affine_dequant_row(d_blob, H, I, d_bits, d_group, r, wrow);
+    for (int j = 0; j < n; ++j) {
+      double acc = 0.0;
+      for (int c = 0; c < I; ++c) acc += wrow[c] * g[(int64_t)j * I + c];
+      ys[(int64_t)j * H + r] = acc;
+    }
+  }
+  free(wrow);
+  free(g);
+  free(u);
+  return 0;
 }
 
 /* The bf16 shared expert [MAP-SH] on n rows: same clamped SwiGLU FFN. */

@@ -86,3 +86,28 @@ def dense_layer(dims, x_bits, router_w, bias, gates, ups, downs, shared=None, to
         wg, wu, wd = (bf16_to_f64(a) for a in shared)
         out += swiglu(x @ wg.T, x @ wu.T, dims.swiglu_limit) @ wd.T
     return out, mask
+
+
+def affine_dequant_dense(blob: np.ndarray, rows: int, cols: int, bits: int, group: int) -> np.ndarray:
+    """Affine low-bit weights w = scale * q + bias, dense fp64 [rows, cols]:
+    the code bit stream unpacked with numpy's little-endian unpackbits and
+    weighted by powers of two (not extracted code by code), scales and biases
+    read as bf16 planes."""
+    cb = rows * cols * bits // 8
+    b = np.asarray(blob, np.uint8)
+    bitsarr = np.unpackbits(b[:cb].reshape(rows, cols * bits // 8), axis=1, bitorder="little")
+    q = (bitsarr.reshape(rows, cols, bits).astype(np.int64) * (1 << np.arange(bits))).sum(axis=2)
+    ng = rows * (cols // group)
+    s = bf16_to_f64(b[cb:cb + 2 * ng].view(np.uint16)).reshape(rows, cols // group)
+    z = bf16_to_f64(b[cb + 2 * ng:cb + 4 * ng].view(np.uint16)).reshape(rows, cols // group)
+    return np.repeat(s, group, axis=1) * q + np.repeat(z, group, axis=1)
+
+
+def affine_pack(q: np.ndarray, scale_bits: np.ndarray, bias_bits: np.ndarray, bits: int) -> np.ndarray:
+    """Blob from codes [rows, cols] (0 .. 2^bits - 1) and bf16 scale / bias
+    bits [rows, cols/G]: each code's bits spread LSB first with packbits."""
+    rows, cols = q.shape
+    bitmat = ((q[:, :, None] >> np.arange(bits)) & 1).astype(np.uint8).reshape(rows, cols * bits)
+    codes = np.packbits(bitmat, axis=1, bitorder="little").reshape(-1)
+    return np.concatenate([codes, np.asarray(scale_bits, np.uint16).reshape(-1).view(np.uint8),
+                           np.asarray(bias_bits, np.uint16).reshape(-1).view(np.uint8)])
